@@ -1,0 +1,84 @@
+// internal.h -- structures shared by the host runtime and the kernels of libsegkv.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace skv {
+
+// Device error codes written to state[1] (first error wins); values match segkv_status.
+constexpr int kErrDeviceBounds = 7;
+constexpr int kErrDeviceTimeout = 8;
+
+// Per-call metadata blobs are uploaded into the head of the caller's workspace with one
+// host-to-device copy.  The first 64 bytes are scheduler counters that the upload zeroes.
+constexpr int kHeaderBytes = 64;
+
+struct AppendSeq {   // one sequence of an append call
+  int32_t seq_id, start, count, tok_off;
+};
+
+struct PrefillSeq {  // one sequence of a prefill call
+  int32_t seq_id, q_start, q_len, q_row0;
+  int32_t kv_len, pad0, pad1, pad2;
+};
+
+struct DecodeSeq {   // one sequence of a decode call
+  int32_t seq_id, q_pos, kv_len, pad;
+};
+
+// A work item is two int32 words: w0 = sequence index in the call,
+// w1 = (global << 31) | (kv_head << 20) | tile_or_split.
+__host__ __device__ inline int item_head(uint32_t w1) { return (int)((w1 >> 20) & 0x7FF); }
+__host__ __device__ inline int item_tile(uint32_t w1) { return (int)(w1 & 0xFFFFF); }
+__host__ __device__ inline bool item_global(uint32_t w1) { return (w1 >> 31) != 0; }
+__host__ __device__ inline uint32_t make_item_w1(bool global, int head, int tile) {
+  return ((uint32_t)global << 31) | ((uint32_t)head << 20) | (uint32_t)tile;
+}
+
+struct StorageGeom {  // what every kernel needs to resolve a logical position to a page
+  int32_t *page_table;
+  const int32_t *free_list;
+  int32_t *state;
+  void *k_pool, *v_pool;
+  int num_pages, page, head_dim, hkv, hq, max_seqs, max_lp, ring, window;
+};
+
+// -- launchers (each .cu file exposes one host function per kernel) --------------------
+cudaError_t launch_reset(const StorageGeom &g, int num_layers, cudaStream_t st);
+
+cudaError_t launch_append(const StorageGeom &g, int layer, const void *ws_meta, int nseq, const uint8_t *cls_dev,
+                          int total_tokens, const void *k_new, const void *v_new, cudaStream_t st);
+
+struct PrefillLaunch {
+  StorageGeom g;
+  int layer, nseq, n_items, tile_pos, grid;
+  const void *ws_meta;  // header + PrefillSeq[nseq] + items
+  int items_off;        // byte offset of the item array inside ws_meta
+  const void *q;
+  void *out;
+  float *lse;
+  unsigned long long *visited;
+  float scale_log2;
+};
+cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                           const CUtensorMap &vmap, cudaStream_t st);
+int prefill_smem_bytes(int head_dim);
+
+struct DecodeLaunch {
+  StorageGeom g;
+  int layer, nseq, n_items, split_pages, max_splits, grid;
+  const void *ws_meta;  // header + DecodeSeq[nseq] + nsplit[nseq*hkv] + items
+  int nsplit_off, items_off;
+  float *part_o, *part_lse;  // [nseq, hq, max_splits, D], [nseq, hq, max_splits]
+  const void *q;
+  void *out;
+  float *lse;
+  unsigned long long *visited;
+  float scale_log2;
+};
+cudaError_t launch_decode(const DecodeLaunch &p, const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t st);
+int decode_smem_bytes(int head_dim);
+
+}  // namespace skv

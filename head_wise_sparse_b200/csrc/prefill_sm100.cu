@@ -1,0 +1,432 @@
+// prefill_sm100.cu -- causal variable-length prefill over per-head paged KV storage,
+// tcgen05 tensor cores with TMEM accumulators, TMA page loads, persistent LPT scheduling
+// (north star subsystems (2) and (4)).
+//
+// What it computes (zhichai.net news item "What Happened", item 3): for every query row of
+// every head, attention over exactly the keys that head keeps, with the head's visibility
+// (global: k <= p; local: p - W < k <= p) decided from positions -- no mask tensor.
+//
+// Structure of one CTA (persistent, one per SM, 192 threads):
+//   warp 0      producer: takes the next item of the longest-first list (atomic counter),
+//               loads the Q tile once, then streams K and V tiles page by page through TMA
+//               (a tile of BN = 128 keys is BN/P pages resolved through the head's page table)
+//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (two S buffers), then
+//               O += P V with P read from TMEM
+//   warps 2..5  softmax: one thread per row of the 128-row tile; fp32 online softmax in the
+//               exp2 domain, rescales O only when the row maximum grows by more than 2^8,
+//               writes P (bf16) back into TMEM over its S buffer, and finally normalises O,
+//               writes bf16 out, fp32 lse and the visited-pair counts.
+// A 128-row tile packs the G query heads of one KV head (GQA group) over 128/G positions.
+#include "device_common.cuh"
+
+namespace skv {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
+constexpr int kColS0 = 0, kColO = 256;     // TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D)
+
+template <int D>
+struct Smem {
+  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kTileBytes = kBN * D * 2;
+  static constexpr int kHalves = D / 64;
+  static constexpr int kBarOff = kQBytes + 2 * kStages * kTileBytes;
+  static constexpr int kBytes = 1024 + kBarOff + 512;
+};
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_ready[2], pv_done[2];
+  uint64_t o_free, mma_done;
+  uint64_t sched_full[4], sched_empty[4];
+  int sched[4];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Item {
+  int b, h, t, npos, q_first, q_last, lo_min, kt_lo, kt_hi, seq_id, kv_len, q_row;
+  bool global;
+};
+
+__device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const PrefillSeq *seqs, const int2 *items,
+                                            int idx) {
+  const int2 w = items[idx];
+  Item it;
+  it.b = w.x;
+  const uint32_t w1 = (uint32_t)w.y;
+  it.h = item_head(w1);
+  it.t = item_tile(w1);
+  it.global = item_global(w1);
+  const PrefillSeq s = seqs[it.b];
+  it.seq_id = s.seq_id;
+  it.kv_len = s.kv_len;
+  it.q_first = s.q_start + it.t * p.tile_pos;
+  it.npos = min(p.tile_pos, s.q_len - it.t * p.tile_pos);
+  it.q_last = it.q_first + it.npos - 1;
+  it.q_row = s.q_row0 + it.t * p.tile_pos;
+  it.lo_min = it.global ? 0 : max(0, it.q_first - p.g.window + 1);
+  it.kt_lo = it.lo_min / kBN;
+  it.kt_hi = it.q_last / kBN;
+  return it;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const PrefillLaunch p) {
+  using S = Smem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *q_s = base;
+  uint8_t *k_s = base + S::kQBytes;
+  uint8_t *v_s = k_s + kStages * S::kTileBytes;
+  Bars *bar = reinterpret_cast<Bars *>(base + S::kBarOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const char *meta = static_cast<const char *>(p.ws_meta);
+  int *sched_next = const_cast<int *>(reinterpret_cast<const int *>(meta));
+  const PrefillSeq *seqs = reinterpret_cast<const PrefillSeq *>(meta + kHeaderBytes);
+  const int2 *items = reinterpret_cast<const int2 *>(meta + p.items_off);
+  const int G = p.g.hq / p.g.hkv;
+  int32_t *state = p.g.state;
+  volatile int *abort_flag = &bar->abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_empty[s], 1);
+      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar->s_full[b], 1);
+      mbar_init(&bar->p_ready[b], 128);
+      mbar_init(&bar->pv_done[b], 1);
+    }
+    mbar_init(&bar->o_free, 128);
+    mbar_init(&bar->mma_done, 1);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&bar->sched_full[s], 1);
+      mbar_init(&bar->sched_empty[s], 5);  // MMA thread + lane 0 of each softmax warp
+    }
+    bar->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&bar->tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+    }
+    const int P = p.g.page, PPT = kBN / P;
+    int i = 0, c = 0;
+    bool ok = true;
+    for (;;) {
+      int idx = 0;
+      if (lane == 0) idx = atomicAdd(sched_next, 1);
+      idx = __shfl_sync(0xffffffffu, idx, 0);
+      if (idx >= p.n_items) idx = -1;
+      const int slot = i & 3;
+      if (!(ok = warp_wait(&bar->sched_empty[slot], ((i >> 2) & 1) ^ 1, abort_flag, state))) break;
+      if (lane == 0) {
+        bar->sched[slot] = idx;
+        mbar_arrive(&bar->sched_full[slot]);
+      }
+      if (idx < 0) break;
+      const Item it = decode_item(p, seqs, items, idx);
+      if (!(ok = warp_wait(&bar->q_empty, (i & 1) ^ 1, abort_flag, state))) break;
+      if (lane == 0) {
+        mbar_expect_tx(&bar->q_full, S::kQBytes);
+        for (int hh = 0; hh < S::kHalves; ++hh)
+          tma_load_3d(q_s + hh * kBM * 128, &qmap, &bar->q_full, hh * 64, it.h * G, it.q_row);
+      }
+      const long long row_base = (((long long)p.layer * p.g.max_seqs + it.seq_id) * p.g.hkv + it.h) * p.g.max_lp;
+      const int last_lp = (it.kv_len - 1) / P;
+      int lp_base = -(1 << 30), pid = p.g.num_pages;
+      for (int kt = it.kt_lo; kt <= it.kt_hi && ok; ++kt) {
+        const int lp_first = kt * PPT;
+        if (lp_first < lp_base || lp_first + PPT > lp_base + 32) {
+          // resolve 32 logical pages at once, one per lane; out-of-range pages load zeros
+          lp_base = lp_first;
+          const int lp = lp_base + lane;
+          pid = p.g.num_pages;
+          const bool stored = lp <= last_lp && (it.global || lp >= last_lp - p.g.ring + 1);
+          if (stored) {
+            const int32_t v = p.g.page_table[row_base + (it.global ? lp : lp % p.g.ring)];
+            if (v >= 0 && v < p.g.num_pages) pid = v;
+            else if ((long long)lp * P + P - 1 >= it.lo_min && lp * P <= it.q_last) set_error(state, kErrDeviceBounds);
+          }
+        }
+        const int s = c % kStages;
+        const uint32_t u = (uint32_t)(c / kStages);
+        if (!(ok = warp_wait(&bar->k_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
+        if (lane == 0) mbar_expect_tx(&bar->k_full[s], S::kTileBytes);
+        for (int j = 0; j < PPT; ++j) {
+          const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
+          if (lane == 0)
+            for (int hh = 0; hh < S::kHalves; ++hh)
+              tma_load_3d(k_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, &kmap, &bar->k_full[s], hh * 64, 0,
+                          phys);
+        }
+        if (!(ok = warp_wait(&bar->v_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
+        if (lane == 0) mbar_expect_tx(&bar->v_full[s], S::kTileBytes);
+        for (int j = 0; j < PPT; ++j) {
+          const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
+          if (lane == 0)
+            for (int hh = 0; hh < S::kHalves; ++hh)
+              tma_load_3d(v_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, &vmap, &bar->v_full[s], hh * 64, 0,
+                          phys);
+        }
+        ++c;
+      }
+      if (!ok) break;
+      ++i;
+    }
+    // drain: no copy of this CTA may still be in flight when it exits
+    for (int k = c - 1; k >= 0 && k >= c - kStages; --k) {
+      const int s = k % kStages;
+      const uint32_t u = (uint32_t)(k / kStages);
+      mbar_wait_drain(&bar->k_full[s], u & 1);
+      mbar_wait_drain(&bar->v_full[s], u & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, 0, 0);
+      constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, 0, 1);
+      const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
+      int i = 0, c = 0;
+      bool ok = true;
+      auto issue_pv = [&](int cc, bool first, int item) -> bool {
+        const int buf = cc & 1, s = cc % kStages;
+        const uint32_t u = (uint32_t)(cc / kStages);
+        if (!mbar_wait(&bar->p_ready[buf], (cc >> 1) & 1, abort_flag, state)) return false;
+        if (!mbar_wait(&bar->v_full[s], u & 1, abort_flag, state)) return false;
+        if (first && !mbar_wait(&bar->o_free, (item & 1) ^ 1, abort_flag, state)) return false;
+        tc_fence_after();
+        const uint32_t vb = v_addr + s * S::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts(tmem + kColO, tmem + kColS0 + buf * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, kBN * 128, 1024),
+                  kIdescPV, (!first || kk > 0) ? 1u : 0u);
+        umma_commit(&bar->pv_done[buf]);
+        umma_commit(&bar->v_empty[s]);
+        return true;
+      };
+      for (;;) {
+        const int slot = i & 3;
+        if (!(ok = mbar_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state))) break;
+        const int idx = bar->sched[slot];
+        mbar_arrive(&bar->sched_empty[slot]);
+        if (idx < 0) break;
+        const Item it = decode_item(p, seqs, items, idx);
+        const int n_tiles = it.kt_hi - it.kt_lo + 1;
+        if (!(ok = mbar_wait(&bar->q_full, i & 1, abort_flag, state))) break;
+        tc_fence_after();
+        for (int j = 0; j < n_tiles; ++j) {
+          const int s = c % kStages, buf = c & 1;
+          const uint32_t u = (uint32_t)(c / kStages);
+          if (!(ok = mbar_wait(&bar->k_full[s], u & 1, abort_flag, state))) break;
+          tc_fence_after();
+          const uint32_t kb = k_addr + s * S::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off_q = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+            const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+            umma_ss(tmem + kColS0 + buf * 128, sdesc_sw128(q_addr + off_q, 16, 1024),
+                    sdesc_sw128(kb + off_k, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar->s_full[buf]);
+          umma_commit(&bar->k_empty[s]);
+          if (j == n_tiles - 1) umma_commit(&bar->q_empty);
+          if (j > 0 && !(ok = issue_pv(c - 1, j == 1, i))) break;
+          ++c;
+        }
+        if (!ok) break;
+        if (!(ok = issue_pv(c - 1, n_tiles == 1, i))) break;
+        ++i;
+      }
+      // every MMA issued by this thread must finish before TMEM is released
+      umma_commit(&bar->mma_done);
+      mbar_wait_drain(&bar->mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
+    const float sl2 = p.scale_log2;
+    int i = 0, c = 0;
+    for (;;) {
+      const int slot = i & 3;
+      if (!warp_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state)) break;
+      const int idx = bar->sched[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->sched_empty[slot]);
+      if (idx < 0) break;
+      const Item it = decode_item(p, seqs, items, idx);
+      const int n_tiles = it.kt_hi - it.kt_lo + 1;
+      const int pos_local = row / G, g = row % G;
+      const bool valid = pos_local < it.npos;
+      const int pq = it.q_first + min(pos_local, it.npos - 1);
+      const int lo = it.global ? 0 : max(0, pq - p.g.window + 1);
+      float m_used = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int buf = c & 1;
+        if (!(ok = warp_wait(&bar->s_full[buf], (c >> 1) & 1, abort_flag, state))) break;
+        tc_fence_after();
+        uint32_t sr[kBN];
+#pragma unroll
+        for (int cc = 0; cc < kBN / 16; ++cc)
+          tmem_ld16(t_lane + kColS0 + buf * 128 + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[cc * 16]));
+        tmem_ld_wait();
+        float *s = reinterpret_cast<float *>(sr);
+        const int k0 = (it.kt_lo + j) * kBN;
+        if (k0 < lo || k0 + kBN - 1 > pq) {
+#pragma unroll
+          for (int jj = 0; jj < kBN; ++jj) {
+            const int kp = k0 + jj;
+            if (kp < lo || kp > pq) s[jj] = -INFINITY;
+          }
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int jj = 1; jj < kBN; ++jj) mx = fmaxf(mx, s[jj]);
+        const float m_new = mx * sl2;  // -inf stays -inf (scale > 0)
+        const bool grow = m_new > m_used + kRescaleThreshold;
+        // O holds sums of earlier tiles scaled by m_used: rows whose maximum grew past the
+        // threshold rescale it.  TMEM loads/stores need the whole warp, so the warp goes
+        // through the loop when any of its rows does, with factor 1 for the others.
+        const bool rescale = grow && m_used != -INFINITY;
+        if (__any_sync(0xffffffffu, rescale)) {
+          const int pc = c - 1;  // the last PV must have landed in O
+          if (!(ok = warp_wait(&bar->pv_done[pc & 1], (pc >> 1) & 1, abort_flag, state))) break;
+          tc_fence_after();
+          const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.0f;
+#pragma unroll
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t o[16];
+            tmem_ld16(t_lane + kColO + cc * 16, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(t_lane + kColO + cc * 16, o);
+          }
+          tmem_st_wait();
+          l *= alpha;
+        }
+        if (grow) m_used = m_new;
+        uint32_t pk[kBN / 2];
+        float rs = 0.f;
+        if (m_used == -INFINITY) {
+#pragma unroll
+          for (int jj = 0; jj < kBN / 2; ++jj) pk[jj] = 0u;
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < kBN / 2; ++jj) {
+            const float a = fast_exp2(fmaf(s[2 * jj], sl2, -m_used));
+            const float b2 = fast_exp2(fmaf(s[2 * jj + 1], sl2, -m_used));
+            rs += a + b2;
+            pk[jj] = pack_bf16x2(a, b2);
+          }
+        }
+        l += rs;
+#pragma unroll
+        for (int cc = 0; cc < kBN / 32; ++cc)
+          tmem_st16(t_lane + kColS0 + buf * 128 + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[cc * 16]));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar->p_ready[buf]);
+        ++c;
+      }
+      if (!ok) break;
+      // epilogue: the last PV of this item
+      const int pc = c - 1;
+      if (!warp_wait(&bar->pv_done[pc & 1], (pc >> 1) & 1, abort_flag, state)) break;
+      tc_fence_after();
+      const float inv_l = (valid && l > 0.f) ? 1.f / l : 0.f;
+      const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
+#pragma unroll
+      for (int cc = 0; cc < D / 16; ++cc) {
+        uint32_t o[16];
+        tmem_ld16(t_lane + kColO + cc * 16, o);
+        tmem_ld_wait();
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (valid) {
+          dst[cc * 2 + 0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[cc * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar->o_free);
+      if (valid) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;
+      if (p.visited) {
+        unsigned long long cnt = valid ? (unsigned long long)(pq - lo + 1) : 0ull;
+        if (G < 32) {
+          for (int off = G; off < 32; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+          if (lane < G) atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + lane], cnt);
+        } else if (cnt) {
+          atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + g], cnt);
+        }
+      }
+      ++i;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+int prefill_smem_bytes(int head_dim) { return head_dim == 64 ? Smem<64>::kBytes : Smem<128>::kBytes; }
+
+cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                           const CUtensorMap &vmap, cudaStream_t st) {
+  static bool attr_set[2] = {false, false};
+  const int smem = prefill_smem_bytes(p.g.head_dim);
+  cudaError_t e;
+  if (p.g.head_dim == 64) {
+    if (!attr_set[0]) {
+      if ((e = cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+        return e;
+      attr_set[0] = true;
+    }
+    prefill_kernel<64><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, p);
+  } else {
+    if (!attr_set[1]) {
+      if ((e = cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+        return e;
+      attr_set[1] = true;
+    }
+    prefill_kernel<128><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace skv

@@ -1,0 +1,544 @@
+// segkv_runtime.cu -- host runtime of libsegkv: the C ABI declared in include/segkv.h.
+//
+// The runtime validates every call before anything is enqueued, keeps the host's view of
+// sequence lengths and pages handed out (enough to reject a call that would overrun the
+// free list or read a key a local head's ring already dropped), builds the per-call
+// metadata (sequence table, longest-processing-time-first work list), uploads it with one
+// host-to-device copy from pinned staging into the caller's workspace, and launches the
+// kernels.  It never allocates device memory.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/segkv.h"
+#include "internal.h"
+
+using namespace skv;
+
+namespace {
+
+constexpr int kPrefillTileRows = 128;  // rows of a prefill tile (G heads x 128/G positions)
+constexpr int kPrefillKeyTile = 128;   // keys of a prefill key tile
+constexpr int kDecodeStageKeys = 64;   // keys of a decode pipeline stage
+constexpr int kMaxSplits = 32;         // most splits one decode head is cut into
+constexpr int kMaxPairs = 8192;        // (sequence, KV head) pairs of one append
+constexpr int kStagingSlots = 4;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map, 128-byte swizzle, inner box of 64 elements (128 bytes).
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+              uint64_t stride2_bytes, uint32_t box1, uint32_t box2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {64, box1, box2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Staging {
+  void *host = nullptr;
+  size_t cap = 0;
+  cudaEvent_t ev = nullptr;
+  bool pending = false;
+};
+
+}  // namespace
+
+struct segkv {
+  segkv_config cfg;
+  std::vector<uint8_t> cls;  // [layers * hkv]
+  std::vector<int32_t> len;  // [layers * max_seqs]
+  int ring = 0, max_lp = 0, G = 0;
+  long long pages_used = 0;
+  Staging slot[kStagingSlots];
+  int next_slot = 0;
+  bool maps_ready = false;
+  CUtensorMap kmap, vmap;
+  int num_sms = 0;
+};
+
+namespace {
+
+StorageGeom geom(const segkv_t *h) {
+  StorageGeom g;
+  g.page_table = h->cfg.page_table;
+  g.free_list = h->cfg.free_list;
+  g.state = h->cfg.state;
+  g.k_pool = h->cfg.k_pool;
+  g.v_pool = h->cfg.v_pool;
+  g.num_pages = h->cfg.num_pages;
+  g.page = h->cfg.page_size;
+  g.head_dim = h->cfg.head_dim;
+  g.hkv = h->cfg.num_kv_heads;
+  g.hq = h->cfg.num_q_heads;
+  g.max_seqs = h->cfg.max_seqs;
+  g.max_lp = h->max_lp;
+  g.ring = h->ring;
+  g.window = h->cfg.window;
+  return g;
+}
+
+// Pages a head holds once its sequence has `n` tokens.
+int held_pages(const segkv_t *h, bool global, int n) {
+  const int full = ceil_div(n, h->cfg.page_size);
+  return global ? full : std::min(full, h->ring);
+}
+
+// Pinned staging slot big enough for `bytes`; waits for the copy that last used it.
+int staging(segkv_t *h, size_t bytes, void **host) {
+  Staging &s = h->slot[h->next_slot];
+  if (s.pending) {
+    if (cudaEventSynchronize(s.ev) != cudaSuccess) return SEGKV_ERR_CUDA;
+    s.pending = false;
+  }
+  if (!s.ev && cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming) != cudaSuccess) return SEGKV_ERR_CUDA;
+  if (s.cap < bytes) {
+    if (s.host) cudaFreeHost(s.host);
+    s.host = nullptr;
+    s.cap = 0;
+    const size_t cap = std::max<size_t>(align_up(bytes, 4096), 64 << 10);
+    if (cudaHostAlloc(&s.host, cap, cudaHostAllocDefault) != cudaSuccess) return SEGKV_ERR_CUDA;
+    s.cap = cap;
+  }
+  *host = s.host;
+  return SEGKV_OK;
+}
+
+int upload(segkv_t *h, void *ws, size_t bytes, cudaStream_t st) {
+  Staging &s = h->slot[h->next_slot];
+  if (cudaMemcpyAsync(ws, s.host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  if (cudaEventRecord(s.ev, st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  s.pending = true;
+  h->next_slot = (h->next_slot + 1) % kStagingSlots;
+  return SEGKV_OK;
+}
+
+int ensure_device_state(segkv_t *h) {
+  if (h->maps_ready) return SEGKV_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SEGKV_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SEGKV_ERR_CUDA;
+  const segkv_config &c = h->cfg;
+  const uint64_t rowb = (uint64_t)c.head_dim * 2, pageb = rowb * c.page_size;
+  if (!make_map(&h->kmap, c.k_pool, c.head_dim, c.page_size, c.num_pages, rowb, pageb, c.page_size, 1) ||
+      !make_map(&h->vmap, c.v_pool, c.head_dim, c.page_size, c.num_pages, rowb, pageb, c.page_size, 1))
+    return SEGKV_ERR_CUDA;
+  h->maps_ready = true;
+  return SEGKV_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Common checks of a call's sequence list.
+int check_seqs(const segkv_t *h, int layer, int nseq, const int32_t *seq_ids) {
+  if (layer < 0 || layer >= h->cfg.num_layers || nseq < 1 || !seq_ids) return SEGKV_ERR_INVALID_ARG;
+  if (nseq > h->cfg.max_seqs) return SEGKV_ERR_INVALID_ARG;
+  std::vector<char> seen(h->cfg.max_seqs, 0);
+  for (int b = 0; b < nseq; ++b) {
+    const int s = seq_ids[b];
+    if (s < 0 || s >= h->cfg.max_seqs || seen[s]) return SEGKV_ERR_INVALID_ARG;
+    seen[s] = 1;
+  }
+  return SEGKV_OK;
+}
+
+// A local head can serve queries [q_lo, q_hi] only while its ring still holds key
+// max(0, q_lo - W + 1): the ring holds the last R logical pages ending at the last token.
+bool ring_covers(const segkv_t *h, int len, int q_lo) {
+  const int P = h->cfg.page_size;
+  const int need = std::max(0, q_lo - h->cfg.window + 1);
+  return need / P >= (len - 1) / P - h->ring + 1;
+}
+
+bool layer_has_local(const segkv_t *h, int layer) {
+  for (int k = 0; k < h->cfg.num_kv_heads; ++k)
+    if (!h->cls[layer * h->cfg.num_kv_heads + k]) return true;
+  return false;
+}
+
+struct PlanItem {
+  int32_t b, h, t, cost;
+};
+
+// Longest-processing-time-first list: enumerate (b, head, tile), cost = key tiles the
+// tile touches, counting sort by cost descending (stable: ties keep enumeration order).
+void plan_prefill_items(const segkv_t *h, int layer, int nseq, const int32_t *q_start, const int32_t *q_len,
+                        std::vector<PlanItem> &out) {
+  const int tile_pos = kPrefillTileRows / h->G, H = h->cfg.num_kv_heads, W = h->cfg.window;
+  std::vector<PlanItem> items;
+  int max_cost = 0;
+  for (int b = 0; b < nseq; ++b)
+    for (int k = 0; k < H; ++k) {
+      const bool global = h->cls[layer * H + k] != 0;
+      for (int t = 0; t * tile_pos < q_len[b]; ++t) {
+        const int q_first = q_start[b] + t * tile_pos;
+        const int q_last = q_start[b] + std::min((t + 1) * tile_pos, q_len[b]) - 1;
+        const int lo = global ? 0 : std::max(0, q_first - W + 1);
+        const int cost = q_last / kPrefillKeyTile - lo / kPrefillKeyTile + 1;
+        items.push_back({b, k, t, cost});
+        max_cost = std::max(max_cost, cost);
+      }
+    }
+  std::vector<int64_t> start(max_cost + 2, 0);
+  for (const PlanItem &it : items) start[it.cost]++;
+  int64_t acc = 0;
+  for (int c = max_cost; c >= 0; --c) {
+    const int64_t n = start[c];
+    start[c] = acc;
+    acc += n;
+  }
+  out.assign(items.size(), PlanItem{0, 0, 0, 0});
+  for (const PlanItem &it : items) out[start[it.cost]++] = it;
+}
+
+}  // namespace
+
+// ============================================================================== C ABI
+extern "C" {
+
+const char *segkv_strerror(int s) {
+  switch (s) {
+    case SEGKV_OK: return "ok";
+    case SEGKV_ERR_INVALID_ARG: return "invalid argument";
+    case SEGKV_ERR_UNSUPPORTED: return "unsupported shape";
+    case SEGKV_ERR_OUT_OF_PAGES: return "out of pages";
+    case SEGKV_ERR_RING_TOO_SMALL: return "local-head ring too small for the requested queries";
+    case SEGKV_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case SEGKV_ERR_CUDA: return "CUDA error";
+    case SEGKV_ERR_DEVICE_BOUNDS: return "device: page id out of range";
+    case SEGKV_ERR_DEVICE_TIMEOUT: return "device: pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int segkv_create(const segkv_config *c, segkv_t **out) {
+  if (!c || !out) return SEGKV_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (c->num_layers < 1 || c->num_q_heads < 1 || c->num_kv_heads < 1 || c->max_seqs < 1 || c->max_seq_len < 1 ||
+      c->window < 1 || c->num_pages < 1 || c->ring_pages < 0 || c->max_chunk < 0 || !c->head_class)
+    return SEGKV_ERR_INVALID_ARG;
+  if (!c->k_pool || !c->v_pool || !c->page_table || !c->free_list || !c->state) return SEGKV_ERR_INVALID_ARG;
+  if (!aligned(c->k_pool, 16) || !aligned(c->v_pool, 16)) return SEGKV_ERR_INVALID_ARG;
+  if (c->num_q_heads % c->num_kv_heads) return SEGKV_ERR_INVALID_ARG;
+  const int G = c->num_q_heads / c->num_kv_heads;
+  if (G > 128 || (G & (G - 1))) return SEGKV_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return SEGKV_ERR_UNSUPPORTED;
+  if (c->page_size != 16 && c->page_size != 32 && c->page_size != 64) return SEGKV_ERR_UNSUPPORTED;
+  if (c->num_kv_heads > 2047 || c->max_seq_len > (1 << 27)) return SEGKV_ERR_UNSUPPORTED;
+  segkv_t *h = new (std::nothrow) segkv();
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  h->cfg = *c;
+  h->G = G;
+  h->max_lp = ceil_div(c->max_seq_len, c->page_size);
+  if (c->ring_pages > 0) {
+    h->ring = std::min(c->ring_pages, h->max_lp);
+  } else {
+    const int chunk = std::max(c->max_chunk, 1);
+    h->ring = std::min(h->max_lp, ceil_div(c->window + chunk - 1, c->page_size) + 1);
+  }
+  h->cls.assign(c->head_class, c->head_class + (size_t)c->num_layers * c->num_kv_heads);
+  for (uint8_t &x : h->cls) x = x ? 1 : 0;
+  h->len.assign((size_t)c->num_layers * c->max_seqs, 0);
+  h->cfg.head_class = nullptr;
+  *out = h;
+  return SEGKV_OK;
+}
+
+void segkv_destroy(segkv_t *h) {
+  if (!h) return;
+  for (Staging &s : h->slot) {
+    if (s.pending) cudaEventSynchronize(s.ev);
+    if (s.ev) cudaEventDestroy(s.ev);
+    if (s.host) cudaFreeHost(s.host);
+  }
+  delete h;
+}
+
+int segkv_ring_pages(const segkv_t *h) { return h ? h->ring : -1; }
+int segkv_max_lp(const segkv_t *h) { return h ? h->max_lp : -1; }
+int segkv_pages_used(const segkv_t *h) { return h ? (int)h->pages_used : -1; }
+
+int segkv_seq_len(const segkv_t *h, int layer, int seq) {
+  if (!h || layer < 0 || layer >= h->cfg.num_layers || seq < 0 || seq >= h->cfg.max_seqs) return -1;
+  return h->len[(size_t)layer * h->cfg.max_seqs + seq];
+}
+
+size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
+  if (!h || max_batch < 1 || max_tokens < 0) return 0;
+  const size_t H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
+  const int tile_pos = kPrefillTileRows / h->G;
+  const size_t app = kHeaderBytes + sizeof(AppendSeq) * max_batch + H;
+  const size_t pre = kHeaderBytes + sizeof(PrefillSeq) * max_batch +
+                     8 * H * ((size_t)ceil_div(max_tokens, tile_pos) + max_batch) + 16;
+  const size_t dec_meta = align_up(kHeaderBytes + sizeof(DecodeSeq) * max_batch + 4 * max_batch * H +
+                                       8 * max_batch * H * kMaxSplits + 16,
+                                   256);
+  const size_t dec = dec_meta + align_up(4 * (size_t)max_batch * Hq * kMaxSplits * D, 256) +
+                     4 * (size_t)max_batch * Hq * kMaxSplits;
+  return align_up(std::max(app, std::max(pre, dec)), 256);
+}
+
+int segkv_reset(segkv_t *h, void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  if (launch_reset(geom(h), h->cfg.num_layers, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SEGKV_ERR_CUDA;
+  std::fill(h->len.begin(), h->len.end(), 0);
+  h->pages_used = 0;
+  return SEGKV_OK;
+}
+
+int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *start_pos,
+                 const int32_t *num_new, const void *k_new, const void *v_new, void *ws, size_t ws_bytes,
+                 void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  int rc = check_seqs(h, layer, nseq, seq_ids);
+  if (rc) return rc;
+  if (!start_pos || !num_new) return SEGKV_ERR_INVALID_ARG;
+  const int H = h->cfg.num_kv_heads;
+  if ((long long)nseq * H > kMaxPairs) return SEGKV_ERR_UNSUPPORTED;
+  long long total = 0, new_pages = 0;
+  for (int b = 0; b < nseq; ++b) {
+    const int s = seq_ids[b];
+    const int cur = h->len[(size_t)layer * h->cfg.max_seqs + s];
+    if (num_new[b] < 0 || start_pos[b] != cur || (long long)cur + num_new[b] > h->cfg.max_seq_len)
+      return SEGKV_ERR_INVALID_ARG;
+    total += num_new[b];
+    for (int k = 0; k < H; ++k) {
+      const bool global = h->cls[layer * H + k] != 0;
+      new_pages += held_pages(h, global, cur + num_new[b]) - held_pages(h, global, cur);
+    }
+  }
+  if (total > (1LL << 30)) return SEGKV_ERR_UNSUPPORTED;
+  if (total > 0 && (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16))) return SEGKV_ERR_INVALID_ARG;
+  if (h->pages_used + new_pages > h->cfg.num_pages) return SEGKV_ERR_OUT_OF_PAGES;
+  const size_t bytes = kHeaderBytes + sizeof(AppendSeq) * nseq + H;
+  if (!ws || !aligned(ws, 256) || ws_bytes < bytes) return SEGKV_ERR_WORKSPACE;
+  if ((rc = ensure_device_state(h))) return rc;
+  void *host = nullptr;
+  if ((rc = staging(h, bytes, &host))) return rc;
+  std::memset(host, 0, kHeaderBytes);
+  AppendSeq *as = reinterpret_cast<AppendSeq *>(static_cast<char *>(host) + kHeaderBytes);
+  int tok = 0;
+  for (int b = 0; b < nseq; ++b) {
+    as[b] = AppendSeq{seq_ids[b], start_pos[b], num_new[b], tok};
+    tok += num_new[b];
+  }
+  uint8_t *cls = reinterpret_cast<uint8_t *>(as + nseq);
+  std::memcpy(cls, &h->cls[(size_t)layer * H], H);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = upload(h, ws, bytes, st))) return rc;
+  const uint8_t *cls_dev = static_cast<const uint8_t *>(ws) + kHeaderBytes + sizeof(AppendSeq) * nseq;
+  if (launch_append(geom(h), layer, ws, nseq, cls_dev, (int)total, k_new, v_new, st) != cudaSuccess)
+    return SEGKV_ERR_CUDA;
+  for (int b = 0; b < nseq; ++b) h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] += num_new[b];
+  h->pages_used += new_pages;
+  return SEGKV_OK;
+}
+
+int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_start_pos, const int32_t *q_len,
+                       int32_t *items_out, int64_t cap, int64_t *n_items, int *tile_pos, int *key_tile) {
+  if (!h || layer < 0 || layer >= h->cfg.num_layers || nseq < 1 || !q_start_pos || !q_len)
+    return SEGKV_ERR_INVALID_ARG;
+  for (int b = 0; b < nseq; ++b)
+    if (q_len[b] < 0 || q_start_pos[b] < 0) return SEGKV_ERR_INVALID_ARG;
+  std::vector<PlanItem> items;
+  plan_prefill_items(h, layer, nseq, q_start_pos, q_len, items);
+  if (n_items) *n_items = (int64_t)items.size();
+  if (tile_pos) *tile_pos = kPrefillTileRows / h->G;
+  if (key_tile) *key_tile = kPrefillKeyTile;
+  if ((int64_t)items.size() > cap || (!items_out && !items.empty())) return SEGKV_ERR_WORKSPACE;
+  for (size_t i = 0; i < items.size(); ++i) {
+    items_out[4 * i + 0] = items[i].b;
+    items_out[4 * i + 1] = items[i].h;
+    items_out[4 * i + 2] = items[i].t;
+    items_out[4 * i + 3] = items[i].cost;
+  }
+  return SEGKV_OK;
+}
+
+int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                       const int32_t *q_len, const void *q, float softmax_scale, void *out, float *lse,
+                       uint64_t *visited, void *ws, size_t ws_bytes, void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  int rc = check_seqs(h, layer, nseq, seq_ids);
+  if (rc) return rc;
+  if (!q_start_pos || !q_len) return SEGKV_ERR_INVALID_ARG;
+  const bool has_local = layer_has_local(h, layer);
+  long long tq = 0;
+  for (int b = 0; b < nseq; ++b) {
+    const int len = h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]];
+    if (q_len[b] < 0 || q_start_pos[b] < 0 || (long long)q_start_pos[b] + q_len[b] > len) return SEGKV_ERR_INVALID_ARG;
+    if (q_len[b] > 0 && has_local && !ring_covers(h, len, q_start_pos[b])) return SEGKV_ERR_RING_TOO_SMALL;
+    tq += q_len[b];
+  }
+  if (tq == 0) return SEGKV_OK;
+  if (tq > (1LL << 30)) return SEGKV_ERR_UNSUPPORTED;
+  if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4)) return SEGKV_ERR_INVALID_ARG;
+  std::vector<PlanItem> items;
+  plan_prefill_items(h, layer, nseq, q_start_pos, q_len, items);
+  const int items_off = (int)align_up(kHeaderBytes + sizeof(PrefillSeq) * nseq, 16);
+  const size_t bytes = items_off + 8 * items.size();
+  if (!ws || !aligned(ws, 256) || ws_bytes < bytes) return SEGKV_ERR_WORKSPACE;
+  if ((rc = ensure_device_state(h))) return rc;
+  void *host = nullptr;
+  if ((rc = staging(h, bytes, &host))) return rc;
+  std::memset(host, 0, items_off);
+  PrefillSeq *ps = reinterpret_cast<PrefillSeq *>(static_cast<char *>(host) + kHeaderBytes);
+  int row0 = 0;
+  for (int b = 0; b < nseq; ++b) {
+    ps[b] = PrefillSeq{seq_ids[b], q_start_pos[b], q_len[b], row0,
+                       h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]], 0, 0, 0};
+    row0 += q_len[b];
+  }
+  int2 *it = reinterpret_cast<int2 *>(static_cast<char *>(host) + items_off);
+  const int H = h->cfg.num_kv_heads;
+  for (size_t i = 0; i < items.size(); ++i)
+    it[i] = make_int2(items[i].b, (int)make_item_w1(h->cls[layer * H + items[i].h] != 0, items[i].h, items[i].t));
+  CUtensorMap qmap;
+  const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads;
+  if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G, kPrefillTileRows / h->G))
+    return SEGKV_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = upload(h, ws, bytes, st))) return rc;
+  PrefillLaunch p;
+  p.g = geom(h);
+  p.layer = layer;
+  p.nseq = nseq;
+  p.n_items = (int)items.size();
+  p.tile_pos = kPrefillTileRows / h->G;
+  p.grid = std::min<int>((int)items.size(), h->num_sms);
+  p.ws_meta = ws;
+  p.items_off = items_off;
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.visited = reinterpret_cast<unsigned long long *>(visited);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (launch_prefill(p, qmap, h->kmap, h->vmap, st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  return SEGKV_OK;
+}
+
+int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,
+                      const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
+                      void *ws, size_t ws_bytes, void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  int rc = check_seqs(h, layer, nseq, seq_ids);
+  if (rc) return rc;
+  if (!q_pos || num_splits < 0) return SEGKV_ERR_INVALID_ARG;
+  if (h->G > 16) return SEGKV_ERR_UNSUPPORTED;
+  if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4)) return SEGKV_ERR_INVALID_ARG;
+  const int P = h->cfg.page_size, H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
+  const bool has_local = layer_has_local(h, layer);
+  long long total_pages = 0;
+  int max_pages = 0;
+  for (int b = 0; b < nseq; ++b) {
+    const int len = h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]];
+    if (q_pos[b] < 0 || q_pos[b] >= len) return SEGKV_ERR_INVALID_ARG;
+    if (has_local && !ring_covers(h, len, q_pos[b])) return SEGKV_ERR_RING_TOO_SMALL;
+    for (int k = 0; k < H; ++k) {
+      const int lo = h->cls[layer * H + k] ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
+      const int n = q_pos[b] / P - lo / P + 1;
+      total_pages += n;
+      max_pages = std::max(max_pages, n);
+    }
+  }
+  if ((rc = ensure_device_state(h))) return rc;
+  // split size in pages: a multiple of the pages of one 64-key stage
+  const int pps = kDecodeStageKeys / P;
+  int split;
+  if (num_splits > 0) {
+    split = ceil_div(max_pages, std::min(num_splits, kMaxSplits));
+  } else {
+    const long long target = std::max<long long>(1, total_pages / (8LL * h->num_sms));
+    split = 1;
+    while (2LL * split <= target && split < 256) split *= 2;
+  }
+  split = std::max(split, ceil_div(max_pages, kMaxSplits));
+  split = ceil_div(split, pps) * pps;
+  const int max_splits = ceil_div(max_pages, split);
+  const int nsplit_off = kHeaderBytes + (int)sizeof(DecodeSeq) * nseq;
+  const int items_off = (int)align_up(nsplit_off + 4 * nseq * H, 16);
+  std::vector<int2> items;
+  std::vector<int32_t> nsplit((size_t)nseq * H);
+  for (int b = 0; b < nseq; ++b)
+    for (int k = 0; k < H; ++k) {
+      const bool global = h->cls[layer * H + k] != 0;
+      const int lo = global ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
+      const int n = ceil_div(q_pos[b] / P - lo / P + 1, split);
+      nsplit[(size_t)b * H + k] = n;
+      for (int s = 0; s < n; ++s) items.push_back(make_int2(b, (int)make_item_w1(global, k, s)));
+    }
+  const size_t meta_bytes = items_off + 8 * items.size();
+  const size_t part_o_off = align_up(meta_bytes, 256);
+  const size_t part_lse_off = part_o_off + align_up(4 * (size_t)nseq * Hq * max_splits * D, 256);
+  const size_t need = part_lse_off + 4 * (size_t)nseq * Hq * max_splits;
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEGKV_ERR_WORKSPACE;
+  void *host = nullptr;
+  if ((rc = staging(h, meta_bytes, &host))) return rc;
+  std::memset(host, 0, items_off);
+  DecodeSeq *ds = reinterpret_cast<DecodeSeq *>(static_cast<char *>(host) + kHeaderBytes);
+  for (int b = 0; b < nseq; ++b)
+    ds[b] = DecodeSeq{seq_ids[b], q_pos[b], h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]], 0};
+  std::memcpy(static_cast<char *>(host) + nsplit_off, nsplit.data(), 4 * nsplit.size());
+  std::memcpy(static_cast<char *>(host) + items_off, items.data(), 8 * items.size());
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = upload(h, ws, meta_bytes, st))) return rc;
+  DecodeLaunch p;
+  p.g = geom(h);
+  p.layer = layer;
+  p.nseq = nseq;
+  p.n_items = (int)items.size();
+  p.split_pages = split;
+  p.max_splits = max_splits;
+  p.grid = std::min<int>((int)items.size(), h->num_sms);
+  p.ws_meta = ws;
+  p.nsplit_off = nsplit_off;
+  p.items_off = items_off;
+  p.part_o = reinterpret_cast<float *>(static_cast<char *>(ws) + part_o_off);
+  p.part_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + part_lse_off);
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.visited = reinterpret_cast<unsigned long long *>(visited);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (launch_decode(p, h->kmap, h->vmap, st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  return SEGKV_OK;
+}
+
+int segkv_device_status(segkv_t *h, void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  if (cudaMemcpyAsync(&word, h->cfg.state + 1, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SEGKV_ERR_CUDA;
+  if (cudaMemsetAsync(h->cfg.state + 1, 0, sizeof(int32_t), st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  return word;
+}
+
+}  // extern "C"

@@ -1,0 +1,174 @@
+/*
+ * segkv.h -- C ABI of libsegkv.so: head-wise segmented paged KV storage and attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method ("RedKnot"): every (layer, KV head) owns its own paged KV storage holding
+ * only the tokens that head needs.  A few "global" heads keep the full causal context;
+ * the "local" majority keep a sliding window of W tokens (zhichai.net news item "What
+ * Happened", items 1 and 3; hysenlabs.com write-up "The Three Core Mechanisms in
+ * Detail", third mechanism: pages and their visibility organised per head and per
+ * segment).  One variable-length attention pass serves every head over its own pages;
+ * no attention mask is ever built.
+ *
+ * Conventions shared by every entry point
+ *   - Positions are 0-based absolute token positions inside a sequence.
+ *   - G = num_q_heads / num_kv_heads; query head h reads KV head h / G.
+ *   - Visibility of a query at position p: global head  k <= p;
+ *                                          local head   p - W < k <= p  (W keys, self included).
+ *   - softmax_scale <= 0 selects 1/sqrt(head_dim).  lse = ln(sum over visible k of
+ *     exp(softmax_scale * q.k)), fp32.
+ *   - bf16 tensors are passed as void* to raw device memory, row-major, contiguous.
+ *   - Streams are cudaStream_t values passed as void* (NULL = legacy default stream).
+ *     Every call only enqueues work on that stream; nothing blocks except
+ *     segkv_device_status.
+ *   - Ownership: the caller owns every device buffer (pools, page table, free list,
+ *     state, workspace, inputs, outputs).  The library owns the host handle, a host
+ *     copy of the head classes, pinned staging for per-call metadata and CUDA events.
+ *     It never calls cudaMalloc.
+ *   - Errors: every int-returning call returns a segkv_status.  On a non-OK return
+ *     nothing was enqueued and no state changed.  Device-side bounds or timeout
+ *     violations set an error word instead (read it with segkv_device_status); kernels
+ *     never trap.
+ *   - A handle is not thread-safe.  Calls on one handle must be issued from one host
+ *     thread, in stream order.
+ */
+#ifndef SEGKV_H_
+#define SEGKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct segkv segkv_t; /* opaque host handle */
+
+typedef enum {
+  SEGKV_OK = 0,
+  SEGKV_ERR_INVALID_ARG = 1,    /* bad pointer, size, position or length */
+  SEGKV_ERR_UNSUPPORTED = 2,    /* shape outside what the kernels implement */
+  SEGKV_ERR_OUT_OF_PAGES = 3,   /* the free list would run out */
+  SEGKV_ERR_RING_TOO_SMALL = 4, /* a local head's ring no longer holds a needed key */
+  SEGKV_ERR_WORKSPACE = 5,      /* workspace too small or misaligned */
+  SEGKV_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
+  SEGKV_ERR_DEVICE_BOUNDS = 7,  /* (device) page id outside the pool, or unallocated */
+  SEGKV_ERR_DEVICE_TIMEOUT = 8  /* (device) a bounded pipeline wait gave up */
+} segkv_status;
+
+typedef struct {
+  int num_layers;
+  int num_q_heads;
+  int num_kv_heads;   /* num_q_heads % num_kv_heads == 0; G = Hq/Hkv in {1,2,4,8,16,32,64,128} */
+  int head_dim;       /* 64 or 128 */
+  int page_size;      /* tokens per page: 16, 32 or 64 */
+  int window;         /* W >= 1, keys a local head sees (self included) */
+  int ring_pages;     /* R: pages of a local head's ring; 0 selects
+                         min(ceil(max_seq_len/P), ceil((W + max_chunk - 1)/P) + 1) */
+  int max_seqs;       /* sequence slots; seq ids are 0..max_seqs-1 */
+  int max_seq_len;    /* longest sequence, tokens */
+  int max_chunk;      /* longest query range of one prefill call (used for the default R) */
+  const uint8_t *head_class; /* HOST [num_layers * num_kv_heads], 1 = global, 0 = local; copied */
+  int num_pages;      /* N: physical pages in each pool */
+  void *k_pool;       /* DEVICE bf16 [N, page_size, head_dim]; 16-byte aligned */
+  void *v_pool;       /* DEVICE bf16 [N, page_size, head_dim]; 16-byte aligned */
+  int32_t *page_table;       /* DEVICE int32 [num_layers, max_seqs, num_kv_heads, max_lp],
+                                max_lp = ceil(max_seq_len / page_size); all -1 initially */
+  const int32_t *free_list;  /* DEVICE int32 [N]: the order in which physical pages are handed out
+                                (normally a permutation of 0..N-1) */
+  int32_t *state;            /* DEVICE int32 [4]: [0] pages handed out, [1] error word; zero initially */
+} segkv_config;
+
+/* Validates the configuration and creates a handle.  Touches no GPU memory.
+ * Returns INVALID_ARG / UNSUPPORTED for bad shapes. */
+int segkv_create(const segkv_config *cfg, segkv_t **out);
+
+/* Frees the host handle and its pinned staging.  Device buffers stay the caller's. */
+void segkv_destroy(segkv_t *h);
+
+/* Effective ring size R and page-table row length max_lp of a handle. */
+int segkv_ring_pages(const segkv_t *h);
+int segkv_max_lp(const segkv_t *h);
+
+/* Tokens appended so far to (layer, seq) -- the host's view, updated at enqueue time. */
+int segkv_seq_len(const segkv_t *h, int layer, int seq);
+
+/* Pages handed out so far (host's view of state[0]). */
+int segkv_pages_used(const segkv_t *h);
+
+/* Bytes of device workspace any call with at most max_batch sequences and at most
+ * max_tokens packed tokens needs.  Workspace must be 256-byte aligned; calls on the
+ * same stream may share one workspace. */
+size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens);
+
+/* Empties every sequence: page table <- -1, state <- 0 (device, enqueued), lengths <- 0 (host). */
+int segkv_reset(segkv_t *h, void *stream);
+
+/*
+ * Appends tokens [start_pos[b], start_pos[b] + num_new[b]) of sequence seq_ids[b] to every
+ * KV head of `layer` (north star subsystem (1): per-head page-table builder and KV
+ * append/scatter).  start_pos[b] must equal segkv_seq_len(h, layer, seq_ids[b]); seq ids
+ * in one call are distinct.  k_new / v_new: DEVICE bf16 [sum(num_new), Hkv, D],
+ * sequences packed in call order.
+ *   Page rule: every unallocated slot touched takes the next id of the free list, in the
+ *   order (sequence in call order, KV head ascending, logical page ascending).  A global
+ *   head stores logical page lp in slot lp; a local head in slot lp mod R and keeps only
+ *   the last R logical pages ending at the call's last token (older tokens of the call
+ *   are skipped: the ring would overwrite them).  The unwritten rows of a page the call
+ *   starts are zeroed.
+ *   Host arrays: seq_ids, start_pos, num_new [nseq].
+ *   Errors: INVALID_ARG (continuity, range, duplicate ids), OUT_OF_PAGES, WORKSPACE.
+ */
+int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *start_pos,
+                 const int32_t *num_new, const void *k_new, const void *v_new, void *ws, size_t ws_bytes,
+                 void *stream);
+
+/*
+ * Causal variable-length prefill over the segmented storage (north star subsystems (2)
+ * and (4)): for every query row and its query head,
+ *   out = sum_visible softmax(scale * q.k) v   (bf16, RNE),  lse (fp32, natural log),
+ *   visited[b, hq] += number of visible (q,k) pairs (u64, may be NULL).
+ * Queries of sequence seq_ids[b] sit at positions [q_start_pos[b], q_start_pos[b] + q_len[b])
+ * and every one of them must already be appended (q_start_pos + q_len <= seq len).
+ * q, out: DEVICE bf16 [sum(q_len), Hq, D] packed in call order; lse: DEVICE fp32
+ * [sum(q_len), Hq].  Host arrays: seq_ids, q_start_pos, q_len [nseq].
+ * Errors: INVALID_ARG, RING_TOO_SMALL (a local head's ring dropped a key some query
+ * needs), WORKSPACE, CUDA.
+ */
+int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                       const int32_t *q_len, const void *q, float softmax_scale, void *out, float *lse,
+                       uint64_t *visited, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Longest-processing-time-first work list the prefill call would run (host only, no GPU).
+ * Item = (b, kv head, query tile, cost); a query tile holds tile_pos = 128 / G consecutive
+ * positions of all G query heads of the KV head; cost = number of key_tile-aligned key
+ * tiles meeting [lo, q_last] (lo = 0 global, max(0, q_first - W + 1) local); order: cost
+ * descending, item index ascending.  items_out: HOST int32 [cap][4].  *n_items receives
+ * the count (also when cap is too small, which returns WORKSPACE).
+ */
+int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_start_pos, const int32_t *q_len,
+                       int32_t *items_out, int64_t cap, int64_t *n_items, int *tile_pos, int *key_tile);
+
+/*
+ * Decode: one query per sequence at position q_pos[b] (already appended), split-K over
+ * the head's visible pages plus a log-sum-exp combine (north star subsystem (3)).
+ * q, out: DEVICE bf16 [nseq, Hq, D]; lse DEVICE fp32 [nseq, Hq]; visited as for prefill.
+ * num_splits: 0 = automatic, else the largest number of splits any head is cut into.
+ */
+int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,
+                      const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronizes `stream`, reads the device error word, clears it and returns it
+ * (SEGKV_OK, SEGKV_ERR_DEVICE_BOUNDS or SEGKV_ERR_DEVICE_TIMEOUT), or SEGKV_ERR_CUDA. */
+int segkv_device_status(segkv_t *h, void *stream);
+
+/* Static description of a status code. */
+const char *segkv_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEGKV_H_ */

@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Benchmark of the segmented paged attention hot path on B200.
+
+One step = one prefill of the Mistral-7B-shaped single-layer workload (L = 8192, Hq 32,
+Hkv 8, D 128, one global KV head, seven local heads with W = 1024, 64-token pages,
+shuffled physical pages): empty the cache, append the 8192 tokens' K/V into every head's
+own pages (page-table build + scatter), and run the causal varlen prefill over those pages.
+Metric: TFLOP/s over visible (q, k) pairs, FLOPs = 4 * D * sum of visible pairs.
+
+The same JSON line carries a ``decode`` object: the batched-decode workload (64 sequences
+at 32K context, Hq 64, Hkv 8, one global head, W = 4096 rings of 65 pages): per step, the
+append of one new token per sequence plus split-K decode and the LSE combine, in KV GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl segkv|reference]
+
+Under torchrun every rank runs its own replica (weak scaling, no collective on the data
+path); rank 0 prints one JSON line with the whole-job throughput (max time over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from head_wise_sparse_b200 import workloads as wl  # noqa: E402
+
+METRIC = "prefill TFLOP/s over visible (q,k) pairs (% BF16 peak); decode KV GB/s (% HBM)"
+PREFILL = "mistral7b_prefill_L8192"
+DECODE = "decode_64x32k"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PREFILL_SOURCES = ["head_wise_sparse_b200/csrc/prefill_sm100.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
+DECODE_SOURCES = ["head_wise_sparse_b200/csrc/decode.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
+
+
+# ---------------------------------------------------------------------------- helpers
+def visible_pairs(w: wl.Workload, layer: int = 0) -> int:
+    """Visible (q, k) pairs of the workload's queries: p + 1 (global head) or min(p + 1, W)."""
+    n = 0
+    for s in w.seqs:
+        p = np.arange(s.q_lo, s.q_hi, dtype=np.int64)
+        glob = int((p + 1).sum())
+        loc = int(np.minimum(p + 1, w.window).sum())
+        for h in range(w.hq):
+            n += glob if w.classes[layer][h // w.group] else loc
+    return n
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK), "fallback"
+
+
+def sources_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(summary: str, paths):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
+    kernel source (the summary records the source hash); else None."""
+    path = os.path.join(ROOT, "profiles", summary)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", text)
+    t = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+    if not m or not t or m.group(1) != sources_hash(paths):
+        return None
+    return float(t.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        self.windows = []
+
+    def mark(self):
+        return time.time()
+
+    def stop(self):
+        if self.p:
+            self.p.terminate()
+            try:
+                self.p.wait(5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(", ") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        return rows
+
+    def summary(self, t0: float, t1: float):
+        rows = self.stop()
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sel, allr = [], []
+        for r in rows:
+            if len(r) < 10 or (self.uuid and self.uuid not in r[1]):
+                continue
+            try:
+                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            allr.append((ts, r))
+            if t0 - 0.05 <= ts <= t1 + 0.05:
+                sel.append(r)
+        if not sel and allr:  # timed region shorter than the sampling period: nearest samples
+            mid = 0.5 * (t0 + t1)
+            sel = [min(allr, key=lambda x: abs(x[0] - mid))[1]]
+        if not sel:
+            return out
+        try:
+            out["sm_mhz"] = statistics.median(float(r[2]) for r in sel)
+            out["sm_max_mhz"] = max(float(r[3]) for r in sel)
+        except ValueError:
+            pass
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in sel:
+            for n, v in zip(names, r[6:10]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        out["reasons"] = sorted(reasons)
+        out["samples"] = len(sel)
+        return out
+
+
+# ---------------------------------------------------------------------------- oracle (CPU)
+def cpu_baseline(w: wl.Workload, budget_s: float, min_s: float):
+    """The fp64 oracle timed on this host's cores over a seeded sample of query rows of the
+    same workload; returns (TFLOP/s over visible pairs, threads, description)."""
+    import oracle as orc
+    from tests.harness import oracle_replay, q_for_call, step_queries
+
+    o = orc.Oracle.for_workload(w)
+    oracle_replay(w, 0, o)
+    ids, qs, ql = step_queries(w)
+    q = q_for_call(w, 0, ids, qs, ql)
+    total_rows = int(sum(ql)) * w.hq
+    rng = np.random.default_rng(12345)
+    order = rng.permutation(total_rows)
+    done, pairs, t_used, batch = 0, 0, 0.0, 256
+    while t_used < min_s and done < total_rows:
+        rows = np.sort(order[done:done + batch]).astype(np.int64)
+        t = time.perf_counter()
+        _, _, cnt = o.attention(0, ids, qs, ql, q, rows=rows)
+        t_used += time.perf_counter() - t
+        pairs += int(cnt.sum())
+        done += len(rows)
+        if t_used > 0 and t_used < min_s:
+            batch = int(min(max(batch, len(rows) * (min_s - t_used) / max(t_used, 1e-3) * 0.5), 8192))
+        if t_used > budget_s:
+            break
+    tflops = 4.0 * w.d * pairs / t_used / 1e12
+    desc = (f"{done} of {total_rows} query rows (seeded uniform sample) of {w.name}, "
+            f"{pairs} visible pairs, {t_used:.1f} s")
+    return tflops, orc.host_threads(), desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle as orc
+    from tests.harness import oracle_replay, q_for_call, step_queries
+
+    w = wl.CONFIGS[PREFILL]
+    o = orc.Oracle.for_workload(w)
+    oracle_replay(w, 0, o)
+    ids, qs, ql = step_queries(w)
+    q = q_for_call(w, 0, ids, qs, ql)
+    rng = np.random.default_rng(54321)
+    total_rows = int(sum(ql)) * w.hq
+    rows_per_step = 256
+    times, pairs = [], 0
+    for step in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(total_rows, rows_per_step, replace=False)).astype(np.int64)
+        t = time.perf_counter()
+        _, _, cnt = o.attention(0, ids, qs, ql, q, rows=rows)
+        dt = time.perf_counter() - t
+        if step >= args.warmup:
+            times.append(dt)
+            pairs += int(cnt.sum())
+    total_t = sum(times)
+    value = 4.0 * w.d * pairs / total_t / 1e12
+    sample = (f"{rows_per_step} seeded random query rows of {w.name} per step "
+              f"({pairs} visible pairs over {args.steps} timed steps)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": PREFILL, "sample": "rows"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": orc.host_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="segkv", choices=["segkv", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from head_wise_sparse_b200.segkv import SegKV
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    pk, pk_src = peaks()
+    stream = torch.cuda.current_stream()
+
+    # ------------------------------------------------------------------ prefill workload
+    w = wl.CONFIGS[PREFILL]
+    L = w.seqs[0].length
+    q_bits = w.q(0, 0, 0, L)
+    k_bits = w.k(0, 0, 0, L)
+    v_bits = w.v(0, 0, 0, L)
+
+    def dev_bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    q_d, k_d, v_d = dev_bf16(q_bits), dev_bf16(k_bits), dev_bf16(v_bits)
+    kv = SegKV(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=w.page, window=w.window,
+               head_class=w.class_array(), num_pages=w.num_pages, free_list=w.free_list(), max_seqs=1,
+               max_seq_len=L, ring_pages=w.ring_pages, max_chunk=L, ws_batch=1, ws_tokens=L, device=dev)
+    out = torch.empty((L, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((L, w.hq), dtype=torch.float32, device=dev)
+    visited = torch.zeros((1, w.hq), dtype=torch.int64, device=dev)
+    flops = 4.0 * w.d * visible_pairs(w)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+
+    def step():
+        kv.handle.reset(stream)
+        kv.append(0, [0], [0], [L], k_d, v_d)
+
+    for _ in range(args.warmup):
+        step()
+        kv.prefill(0, [0], [0], [L], q_d, out=out, lse=lse, visited=visited)
+    torch.cuda.synchronize()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(str(getattr(props, "uuid", "")))
+    time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    visited.zero_()
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)  # evict L2 between timed steps (not timed)
+        ev[s][0].record(stream)
+        step()
+        ev[s][1].record(stream)
+        kv.prefill(0, [0], [0], [L], q_d, out=out, lse=lse, visited=visited)
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    pre_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    app_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    # the kernel's own count of visited pairs must equal the closed form
+    vis_total = int(visited.sum().item())
+    if vis_total != args.steps * visible_pairs(w):
+        raise RuntimeError(f"visited pairs {vis_total} != {args.steps} x {visible_pairs(w)}")
+    t_step = max_over_ranks(sum(step_ms) / args.steps)
+    t_pre = max_over_ranks(sum(pre_ms) / args.steps)
+    value = world * flops / (t_step * 1e-3) / 1e12
+    achieved = flops / (t_pre * 1e-3) / 1e12
+    traffic = profiled_traffic("prefill_mistral7b_L8192.md", PREFILL_SOURCES)
+
+    # ------------------------------------------------------------------ e2e through host buffers
+    q_h = torch.from_numpy(q_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    k_h = torch.from_numpy(k_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    v_h = torch.from_numpy(v_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_h = torch.empty_like(out, device="cpu").pin_memory()
+    lse_h = torch.empty_like(lse, device="cpu").pin_memory()
+    e2e_steps = min(args.steps, 30)
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for s in range(e2e_steps):
+        flush.fill_(s & 0xFF)
+        ev2[s][0].record(stream)
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        step()
+        kv.prefill(0, [0], [0], [L], q_d, out=out, lse=lse, visited=visited)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        ev2[s][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_e2e = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2) / e2e_steps)
+    h2d = q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    e2e = {"value": world * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e}
+    del kv, flush
+    torch.cuda.empty_cache()
+
+    # ------------------------------------------------------------------ decode workload
+    decode = None
+    if not args.no_decode:
+        decode = bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": PREFILL, "seq_len": L, "q_heads": w.hq, "kv_heads": w.hkv, "head_dim": w.d,
+                   "page_size": w.page, "window": w.window, "global_kv_heads": int(sum(w.classes[0])),
+                   "visible_pairs": visible_pairs(w), "step": "reset + append (page build, scatter) + prefill",
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world}"},
+        "prefill_kernel_ms": t_pre, "append_ms": max_over_ranks(sum(app_ms) / args.steps),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                     "peak_source": f"{pk_src} bf16 burst",
+                     "kernel": "prefill_kernel<128> (events around segkv_prefill_attn: metadata upload + kernel)"},
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if decode is not None:
+        line["decode"] = decode
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v_cpu, cores, desc = cpu_baseline(w, budget_s=3 * args.cpu_seconds, min_s=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk):
+    """Batched decode: 64 sequences, context 32767 (+1 new token per step), split-K + combine."""
+    from head_wise_sparse_b200.segkv import SegKV
+
+    w = wl.CONFIGS[DECODE]
+    B = len(w.seqs)
+    ctx = w.seqs[0].context
+    steps = min(args.steps, 100)
+    warm = args.warmup
+    max_len = ctx + steps + warm + 64
+    wmax = w.scaled(seqs=tuple(wl.Seq(ctx, steps + warm + 1, ctx, ctx + 1) for _ in range(B)))
+    kv = SegKV(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=w.page, window=w.window,
+               head_class=w.class_array(), num_pages=wmax.num_pages, free_list=wmax.free_list(), max_seqs=B,
+               max_seq_len=max_len, ring_pages=w.ring_pages, max_chunk=1, ws_batch=B, ws_tokens=B * 2048, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+    chunk = 2048
+    ids = list(range(B))
+    for lo in range(0, ctx, chunk):
+        n = min(chunk, ctx - lo)
+        k = torch.randn((B * n, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+        v = torch.randn((B * n, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+        kv.append(0, ids, [lo] * B, [n] * B, k, v)
+        del k, v
+    nsteps = warm + steps
+    k_new = torch.randn((nsteps, B, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    v_new = torch.randn((nsteps, B, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn((nsteps, B, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((B, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, w.hq), dtype=torch.float32, device=dev)
+    n_glob = int(sum(w.classes[0]))
+
+    def kv_bytes(p):  # algorithmic KV bytes of one decode step with the query at position p
+        keys = n_glob * (p + 1) + (w.hkv - n_glob) * min(p + 1, w.window)
+        return B * keys * w.d * 2 * 2
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    total_bytes = 0
+    for s in range(nsteps):
+        p = ctx + s
+        timed = s >= warm
+        if timed and s == warm:
+            barrier()
+            torch.cuda.synchronize()
+        if timed:
+            ev[s - warm][0].record(stream)
+        kv.append(0, ids, [p] * B, [1] * B, k_new[s], v_new[s])
+        if timed:
+            ev[s - warm][1].record(stream)
+        kv.decode(0, ids, [p] * B, q[s], out=out, lse=lse)
+        if timed:
+            ev[s - warm][2].record(stream)
+            total_bytes += kv_bytes(p)
+    torch.cuda.synchronize()
+    barrier()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during decode")
+    t_step = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in ev) / steps)
+    t_dec = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / steps)
+    per_step = total_bytes / steps
+    achieved = per_step / (t_dec * 1e-3) / 1e9
+    res = {
+        "workload": DECODE, "metric": "decode KV GB/s", "value": world * per_step / (t_step * 1e-3) / 1e9,
+        "unit": "GB/s", "ms_per_step": t_step, "decode_kernel_ms": t_dec, "steps": steps,
+        "kv_bytes_per_step": per_step, "step": "append 1 token/seq (page build + scatter) + split-K decode + combine",
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic("decode_64x32k.md", DECODE_SOURCES),
+                     "kernel": "decode_split_kernel<128> + lse_combine (events around segkv_decode_attn)"},
+        "gpu_launches": 4 * steps, "data": "synthetic (seeded torch generator on the device)",
+    }
+    del kv
+    torch.cuda.empty_cache()
+    return res
+
+
+if __name__ == "__main__":
+    sys.exit(main())

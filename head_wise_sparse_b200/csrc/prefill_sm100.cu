@@ -6,44 +6,53 @@
 // every head, attention over exactly the keys that head keeps, with the head's visibility
 // (global: k <= p; local: p - W < k <= p) decided from positions -- no mask tensor.
 //
-// Structure of one CTA (persistent, one per SM, 192 threads):
+// Work item = two 128-row query tiles of one (sequence, KV head): each tile packs the G
+// query heads of the KV head over 128/G consecutive positions (GQA group packing), and the
+// two tiles cover 256/G consecutive positions.  Both tiles share every K/V tile load.
+//
+// One persistent CTA per SM, 320 threads:
 //   warp 0      producer: takes the next item of the longest-first list (atomic counter),
-//               loads the Q tile once, then streams K and V tiles page by page through TMA
+//               loads both Q tiles once, then streams K and V tiles page by page through TMA
 //               (a tile of BN = 128 keys is BN/P pages resolved through the head's page table)
-//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (two S buffers), then
-//               O += P V with P read from TMEM
-//   warps 2..5  softmax: one thread per row of the 128-row tile; fp32 online softmax in the
-//               exp2 domain, rescales O only when the row maximum grows by more than 2^8,
-//               writes P (bf16) back into TMEM over its S buffer, and finally normalises O,
-//               writes bf16 out, fp32 lse and the visited-pair counts.
-// A 128-row tile packs the G query heads of one KV head (GQA group) over 128/G positions.
+//   warp 1      MMA issuer (one thread): for key tile j, per query tile t,
+//               O_t += P_t(j-1) V(j-1) then S_t(j) = Q_t K(j)^T, all into TMEM
+//   warps 2..5  softmax of query tile 0, warps 6..9 softmax of query tile 1: one thread per
+//               row; fp32 online softmax in the exp2 domain, O rescaled only when the row
+//               maximum grows by more than 2^8; P (bf16) overwrites its S columns in TMEM;
+//               the epilogue normalises O and writes bf16 out, fp32 lse and visited counts.
+// The two query tiles' chains (S -> softmax -> PV -> next S) interleave on the tensor core:
+// while one tile's warpgroup runs its softmax, the other tile's MMAs run.
 #include "device_common.cuh"
 
 namespace skv {
 
 namespace {
 
-constexpr int kBM = 128;
-constexpr int kBN = 128;
-constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kTileRows = 128;  // rows of one query tile (one TMEM accumulator)
+constexpr int kBN = 128;        // keys of one key tile
+constexpr int kStages = 2;      // K and V ring depth
+constexpr int kThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
-constexpr int kColS0 = 0, kColO = 256;     // TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D)
 
 template <int D>
 struct Smem {
-  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kQTileBytes = kTileRows * D * 2;
   static constexpr int kTileBytes = kBN * D * 2;
   static constexpr int kHalves = D / 64;
-  static constexpr int kBarOff = kQBytes + 2 * kStages * kTileBytes;
+  static constexpr int kKOff = 2 * kQTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   static constexpr int kBytes = 1024 + kBarOff + 512;
+  // TMEM columns: S_t at 128 t, O_t at 256 + 128 t
+  static constexpr uint32_t col_s(int t) { return 128u * t; }
+  static constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
 };
 
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_ready[2], pv_done[2];
-  uint64_t o_free, mma_done;
+  uint64_t s_full[2], p_ready[2], pv_done[2], o_free[2];
+  uint64_t mma_done;
   uint64_t sched_full[4], sched_empty[4];
   int sched[4];
   uint32_t tmem_base;
@@ -51,10 +60,12 @@ struct Bars {
 };
 
 struct Item {
-  int b, h, t, npos, q_first, q_last, lo_min, kt_lo, kt_hi, seq_id, kv_len, q_row;
+  int b, h, t, q_first, q_last, lo_min, kt_lo, kt_hi, seq_id, kv_len, q_row;
   bool global;
 };
 
+// Item = (sequence b, KV head h, tile pair t): positions [q_start + 2 t tp, ...) of the
+// sequence's queries, tp = 128 / G positions per query tile.
 __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const PrefillSeq *seqs, const int2 *items,
                                             int idx) {
   const int2 w = items[idx];
@@ -65,12 +76,12 @@ __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const Prefil
   it.t = item_tile(w1);
   it.global = item_global(w1);
   const PrefillSeq s = seqs[it.b];
+  const int pair = 2 * p.tile_pos;
   it.seq_id = s.seq_id;
   it.kv_len = s.kv_len;
-  it.q_first = s.q_start + it.t * p.tile_pos;
-  it.npos = min(p.tile_pos, s.q_len - it.t * p.tile_pos);
-  it.q_last = it.q_first + it.npos - 1;
-  it.q_row = s.q_row0 + it.t * p.tile_pos;
+  it.q_first = s.q_start + it.t * pair;
+  it.q_last = s.q_start + min((it.t + 1) * pair, s.q_len) - 1;
+  it.q_row = s.q_row0 + it.t * pair;
   it.lo_min = it.global ? 0 : max(0, it.q_first - p.g.window + 1);
   it.kt_lo = it.lo_min / kBN;
   it.kt_hi = it.q_last / kBN;
@@ -78,15 +89,15 @@ __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const Prefil
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(200)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const PrefillLaunch p) {
   using S = Smem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_s = base;
-  uint8_t *k_s = base + S::kQBytes;
-  uint8_t *v_s = k_s + kStages * S::kTileBytes;
+  uint8_t *k_s = base + S::kKOff;
+  uint8_t *v_s = base + S::kVOff;
   Bars *bar = reinterpret_cast<Bars *>(base + S::kBarOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,16 +118,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar->v_full[s], 1);
       mbar_init(&bar->v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bar->s_full[b], 1);
-      mbar_init(&bar->p_ready[b], 128);
-      mbar_init(&bar->pv_done[b], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar->s_full[t], 1);
+      mbar_init(&bar->p_ready[t], 128);
+      mbar_init(&bar->pv_done[t], 1);
+      mbar_init(&bar->o_free[t], 128);
     }
-    mbar_init(&bar->o_free, 128);
     mbar_init(&bar->mma_done, 1);
     for (int s = 0; s < 4; ++s) {
       mbar_init(&bar->sched_full[s], 1);
-      mbar_init(&bar->sched_empty[s], 5);  // MMA thread + lane 0 of each softmax warp
+      mbar_init(&bar->sched_empty[s], 9);  // MMA thread + lane 0 of each of the 8 softmax warps
     }
     bar->abort_flag = 0;
     fence_mbar_init();
@@ -136,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int P = p.g.page, PPT = kBN / P;
     int i = 0, c = 0;
-    bool ok = true;
+    bool ok = true, q_loaded = false;
     for (;;) {
       int idx = 0;
       if (lane == 0) idx = atomicAdd(sched_next, 1);
@@ -152,17 +163,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = decode_item(p, seqs, items, idx);
       if (!(ok = warp_wait(&bar->q_empty, (i & 1) ^ 1, abort_flag, state))) break;
       if (lane == 0) {
-        mbar_expect_tx(&bar->q_full, S::kQBytes);
-        for (int hh = 0; hh < S::kHalves; ++hh)
-          tma_load_3d(q_s + hh * kBM * 128, &qmap, &bar->q_full, hh * 64, it.h * G, it.q_row);
+        mbar_expect_tx(&bar->q_full, 2 * S::kQTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            tma_load_3d(q_s + t * S::kQTileBytes + hh * kTileRows * 128, &qmap, &bar->q_full, hh * 64, it.h * G,
+                        it.q_row + t * p.tile_pos);
       }
+      q_loaded = true;
       const long long row_base = (((long long)p.layer * p.g.max_seqs + it.seq_id) * p.g.hkv + it.h) * p.g.max_lp;
       const int last_lp = (it.kv_len - 1) / P;
       int lp_base = -(1 << 30), pid = p.g.num_pages;
-      for (int kt = it.kt_lo; kt <= it.kt_hi && ok; ++kt) {
+      for (int kt = it.kt_lo; kt <= it.kt_hi; ++kt) {
         const int lp_first = kt * PPT;
         if (lp_first < lp_base || lp_first + PPT > lp_base + 32) {
-          // resolve 32 logical pages at once, one per lane; out-of-range pages load zeros
+          // resolve 32 logical pages at once, one per lane; pages not stored load zeros
           lp_base = lp_first;
           const int lp = lp_base + lane;
           pid = p.g.num_pages;
@@ -205,29 +219,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(&bar->k_full[s], u & 1);
       mbar_wait_drain(&bar->v_full[s], u & 1);
     }
+    if (q_loaded) mbar_wait_drain(&bar->q_full, (uint32_t)((ok ? i - 1 : i) & 1));
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, 0, 0);
-      constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, 0, 1);
+      constexpr uint32_t kIdescQK = idesc_bf16(kTileRows, kBN, 0, 0);
+      constexpr uint32_t kIdescPV = idesc_bf16(kTileRows, D, 0, 1);
       const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
       int i = 0, c = 0;
       bool ok = true;
-      auto issue_pv = [&](int cc, bool first, int item) -> bool {
-        const int buf = cc & 1, s = cc % kStages;
-        const uint32_t u = (uint32_t)(cc / kStages);
-        if (!mbar_wait(&bar->p_ready[buf], (cc >> 1) & 1, abort_flag, state)) return false;
-        if (!mbar_wait(&bar->v_full[s], u & 1, abort_flag, state)) return false;
-        if (first && !mbar_wait(&bar->o_free, (item & 1) ^ 1, abort_flag, state)) return false;
+      // O_t += P_t(cc) V(cc); the first PV of an item overwrites O_t
+      auto issue_pv = [&](int t, int cc, bool first) -> bool {
+        const int s = cc % kStages;
+        if (!mbar_wait(&bar->p_ready[t], cc & 1, abort_flag, state)) return false;
+        if (t == 0 && !mbar_wait(&bar->v_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
+        if (first && !mbar_wait(&bar->o_free[t], (i & 1) ^ 1, abort_flag, state)) return false;
         tc_fence_after();
         const uint32_t vb = v_addr + s * S::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tmem + kColO, tmem + kColS0 + buf * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, kBN * 128, 1024),
+          umma_ts(tmem + S::col_o(t), tmem + S::col_s(t) + kk * 8, sdesc_sw128(vb + kk * 2048, kBN * 128, 1024),
                   kIdescPV, (!first || kk > 0) ? 1u : 0u);
-        umma_commit(&bar->pv_done[buf]);
-        umma_commit(&bar->v_empty[s]);
+        umma_commit(&bar->pv_done[t]);
         return true;
+      };
+      // S_t(cc) = Q_t K(cc)^T
+      auto issue_s = [&](int t, int cc) {
+        const uint32_t kb = k_addr + (cc % kStages) * S::kTileBytes;
+        const uint32_t qb = q_addr + t * S::kQTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off_q = (kk >> 2) * (kTileRows * 128) + (kk & 3) * 32;
+          const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+          umma_ss(tmem + S::col_s(t), sdesc_sw128(qb + off_q, 16, 1024), sdesc_sw128(kb + off_k, 16, 1024),
+                  kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar->s_full[t]);
       };
       for (;;) {
         const int slot = i & 3;
@@ -238,28 +265,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = decode_item(p, seqs, items, idx);
         const int n_tiles = it.kt_hi - it.kt_lo + 1;
         if (!(ok = mbar_wait(&bar->q_full, i & 1, abort_flag, state))) break;
-        tc_fence_after();
-        for (int j = 0; j < n_tiles; ++j) {
-          const int s = c % kStages, buf = c & 1;
-          const uint32_t u = (uint32_t)(c / kStages);
-          if (!(ok = mbar_wait(&bar->k_full[s], u & 1, abort_flag, state))) break;
+        for (int j = 0; j < n_tiles && ok; ++j) {
+          const int s = c % kStages;
+          if (!(ok = mbar_wait(&bar->k_full[s], (uint32_t)(c / kStages) & 1, abort_flag, state))) break;
           tc_fence_after();
-          const uint32_t kb = k_addr + s * S::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off_q = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-            const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-            umma_ss(tmem + kColS0 + buf * 128, sdesc_sw128(q_addr + off_q, 16, 1024),
-                    sdesc_sw128(kb + off_k, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+          for (int t = 0; t < 2; ++t) {
+            if (j > 0 && !(ok = issue_pv(t, c - 1, j == 1))) break;
+            issue_s(t, c);
           }
-          umma_commit(&bar->s_full[buf]);
+          if (!ok) break;
           umma_commit(&bar->k_empty[s]);
+          if (j > 0) umma_commit(&bar->v_empty[(c - 1) % kStages]);
           if (j == n_tiles - 1) umma_commit(&bar->q_empty);
-          if (j > 0 && !(ok = issue_pv(c - 1, j == 1, i))) break;
           ++c;
         }
         if (!ok) break;
-        if (!(ok = issue_pv(c - 1, n_tiles == 1, i))) break;
+        for (int t = 0; t < 2 && ok; ++t) ok = issue_pv(t, c - 1, n_tiles == 1);
+        if (!ok) break;
+        umma_commit(&bar->v_empty[(c - 1) % kStages]);
         ++i;
       }
       // every MMA issued by this thread must finish before TMEM is released
@@ -268,9 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax / epilogue
-    const int q4 = warp & 3;
+    const int tq = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int q4 = warp & 3;         // TMEM lane quadrant of this warp
     const int row = q4 * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t t_s = t_lane + S::col_s(tq), t_o = t_lane + S::col_o(tq);
     const float sl2 = p.scale_log2;
     int i = 0, c = 0;
     for (;;) {
@@ -282,22 +307,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (idx < 0) break;
       const Item it = decode_item(p, seqs, items, idx);
       const int n_tiles = it.kt_hi - it.kt_lo + 1;
-      const int pos_local = row / G, g = row % G;
-      const bool valid = pos_local < it.npos;
-      const int pq = it.q_first + min(pos_local, it.npos - 1);
+      const int pos_local = tq * p.tile_pos + row / G, g = row % G;
+      const int p_raw = it.q_first + pos_local;
+      const bool valid = p_raw <= it.q_last;
+      const int pq = min(p_raw, it.q_last);  // rows past the sequence repeat its last query
       const int lo = it.global ? 0 : max(0, pq - p.g.window + 1);
       float m_used = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
-        const int buf = c & 1;
-        if (!(ok = warp_wait(&bar->s_full[buf], (c >> 1) & 1, abort_flag, state))) break;
+        if (!(ok = warp_wait(&bar->s_full[tq], c & 1, abort_flag, state))) break;
         tc_fence_after();
-        uint32_t sr[kBN];
+        float s[kBN];
 #pragma unroll
         for (int cc = 0; cc < kBN / 16; ++cc)
-          tmem_ld16(t_lane + kColS0 + buf * 128 + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[cc * 16]));
+          tmem_ld16(t_s + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[cc * 16]));
         tmem_ld_wait();
-        float *s = reinterpret_cast<float *>(sr);
         const int k0 = (it.kt_lo + j) * kBN;
         if (k0 < lo || k0 + kBN - 1 > pq) {
 #pragma unroll
@@ -306,60 +330,60 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (kp < lo || kp > pq) s[jj] = -INFINITY;
           }
         }
-        float mx = s[0];
+        float mx8[8];
 #pragma unroll
-        for (int jj = 1; jj < kBN; ++jj) mx = fmaxf(mx, s[jj]);
+        for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+#pragma unroll
+        for (int jj = 8; jj < kBN; jj += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], s[jj + e]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = mx * sl2;  // -inf stays -inf (scale > 0)
         const bool grow = m_new > m_used + kRescaleThreshold;
-        // O holds sums of earlier tiles scaled by m_used: rows whose maximum grew past the
-        // threshold rescale it.  TMEM loads/stores need the whole warp, so the warp goes
-        // through the loop when any of its rows does, with factor 1 for the others.
+        // O_t holds earlier tiles' sums scaled by m_used.  The PV that last wrote it has
+        // completed: it was issued before this tile's S, whose completion we waited for.
+        // TMEM loads/stores need the whole warp, so the warp rescales when any row must,
+        // with factor 1 for the others.
         const bool rescale = grow && m_used != -INFINITY;
         if (__any_sync(0xffffffffu, rescale)) {
-          const int pc = c - 1;  // the last PV must have landed in O
-          if (!(ok = warp_wait(&bar->pv_done[pc & 1], (pc >> 1) & 1, abort_flag, state))) break;
-          tc_fence_after();
           const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.0f;
 #pragma unroll
           for (int cc = 0; cc < D / 16; ++cc) {
             uint32_t o[16];
-            tmem_ld16(t_lane + kColO + cc * 16, o);
+            tmem_ld16(t_o + cc * 16, o);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16(t_lane + kColO + cc * 16, o);
+            tmem_st16(t_o + cc * 16, o);
           }
-          tmem_st_wait();
           l *= alpha;
         }
         if (grow) m_used = m_new;
-        uint32_t pk[kBN / 2];
-        float rs = 0.f;
-        if (m_used == -INFINITY) {
+        // P = exp2(s * scale_log2 - m_used), written as bf16 pairs over the S columns
+        const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int jj = 0; jj < kBN / 2; ++jj) pk[jj] = 0u;
-        } else {
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int jj = 0; jj < kBN / 2; ++jj) {
-            const float a = fast_exp2(fmaf(s[2 * jj], sl2, -m_used));
-            const float b2 = fast_exp2(fmaf(s[2 * jj + 1], sl2, -m_used));
-            rs += a + b2;
-            pk[jj] = pack_bf16x2(a, b2);
+          for (int e = 0; e < 16; ++e) {
+            const float a = fast_exp2(fmaf(s[cc * 32 + 2 * e], sl2, neg_m));
+            const float b2 = fast_exp2(fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m));
+            rs[e & 3] += a + b2;
+            pk[e] = pack_bf16x2(a, b2);
           }
+          tmem_st16(t_s + cc * 16, pk);
         }
-        l += rs;
-#pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc)
-          tmem_st16(t_lane + kColS0 + buf * 128 + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[cc * 16]));
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bar->p_ready[buf]);
+        mbar_arrive(&bar->p_ready[tq]);
         ++c;
       }
       if (!ok) break;
-      // epilogue: the last PV of this item
-      const int pc = c - 1;
-      if (!warp_wait(&bar->pv_done[pc & 1], (pc >> 1) & 1, abort_flag, state)) break;
+      // epilogue: the item's last PV into O_t
+      if (!warp_wait(&bar->pv_done[tq], (c - 1) & 1, abort_flag, state)) break;
       tc_fence_after();
       const float inv_l = (valid && l > 0.f) ? 1.f / l : 0.f;
       const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
@@ -367,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < D / 16; ++cc) {
         uint32_t o[16];
-        tmem_ld16(t_lane + kColO + cc * 16, o);
+        tmem_ld16(t_o + cc * 16, o);
         tmem_ld_wait();
         uint32_t w[8];
 #pragma unroll
@@ -379,13 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&bar->o_free);
+      mbar_arrive(&bar->o_free[tq]);
       if (valid) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;
       if (p.visited) {
         unsigned long long cnt = valid ? (unsigned long long)(pq - lo + 1) : 0ull;
         if (G < 32) {
           for (int off = G; off < 32; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-          if (lane < G) atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + lane], cnt);
+          if (lane < G && cnt) atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + lane], cnt);
         } else if (cnt) {
           atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + g], cnt);
         }

@@ -21,7 +21,8 @@ using namespace skv;
 
 namespace {
 
-constexpr int kPrefillTileRows = 128;  // rows of a prefill tile (G heads x 128/G positions)
+constexpr int kPrefillTileRows = 128;  // rows of one prefill query tile (G heads x 128/G positions)
+constexpr int kPrefillItemRows = 256;  // rows of one prefill work item (two query tiles)
 constexpr int kPrefillKeyTile = 128;   // keys of a prefill key tile
 constexpr int kDecodeStageKeys = 64;   // keys of a decode pipeline stage
 constexpr int kMaxSplits = 32;         // most splits one decode head is cut into
@@ -186,7 +187,7 @@ struct PlanItem {
 // tile touches, counting sort by cost descending (stable: ties keep enumeration order).
 void plan_prefill_items(const segkv_t *h, int layer, int nseq, const int32_t *q_start, const int32_t *q_len,
                         std::vector<PlanItem> &out) {
-  const int tile_pos = kPrefillTileRows / h->G, H = h->cfg.num_kv_heads, W = h->cfg.window;
+  const int tile_pos = kPrefillItemRows / h->G, H = h->cfg.num_kv_heads, W = h->cfg.window;
   std::vector<PlanItem> items;
   int max_cost = 0;
   for (int b = 0; b < nseq; ++b)
@@ -288,7 +289,7 @@ int segkv_seq_len(const segkv_t *h, int layer, int seq) {
 size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
   if (!h || max_batch < 1 || max_tokens < 0) return 0;
   const size_t H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
-  const int tile_pos = kPrefillTileRows / h->G;
+  const int tile_pos = kPrefillItemRows / h->G;
   const size_t app = kHeaderBytes + sizeof(AppendSeq) * max_batch + H;
   const size_t pre = kHeaderBytes + sizeof(PrefillSeq) * max_batch +
                      8 * H * ((size_t)ceil_div(max_tokens, tile_pos) + max_batch) + 16;
@@ -366,7 +367,7 @@ int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_s
   std::vector<PlanItem> items;
   plan_prefill_items(h, layer, nseq, q_start_pos, q_len, items);
   if (n_items) *n_items = (int64_t)items.size();
-  if (tile_pos) *tile_pos = kPrefillTileRows / h->G;
+  if (tile_pos) *tile_pos = kPrefillItemRows / h->G;
   if (key_tile) *key_tile = kPrefillKeyTile;
   if ((int64_t)items.size() > cap || (!items_out && !items.empty())) return SEGKV_ERR_WORKSPACE;
   for (size_t i = 0; i < items.size(); ++i) {

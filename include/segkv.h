@@ -141,7 +141,7 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
 
 /*
  * Longest-processing-time-first work list the prefill call would run (host only, no GPU).
- * Item = (b, kv head, query tile, cost); a query tile holds tile_pos = 128 / G consecutive
+ * Item = (b, kv head, query tile, cost); a query tile holds tile_pos = 256 / G consecutive
  * positions of all G query heads of the KV head; cost = number of key_tile-aligned key
  * tiles meeting [lo, q_last] (lo = 0 global, max(0, q_first - W + 1) local); order: cost
  * descending, item index ascending.  items_out: HOST int32 [cap][4].  *n_items receives

@@ -10,13 +10,15 @@
 // query heads of the KV head over 128/G consecutive positions (GQA group packing), and the
 // two tiles cover 256/G consecutive positions.  Both tiles share every K/V tile load.
 //
-// One persistent CTA per SM, 320 threads:
+// One persistent CTA per SM, 384 threads (three warpgroups; one warp of each per SM
+// sub-partition, so the softmax warps can hold a 128-column S row in registers):
 //   warp 0      producer: takes the next item of the longest-first list (atomic counter),
 //               loads both Q tiles once, then streams K and V tiles page by page through TMA
 //               (a tile of BN = 128 keys is BN/P pages resolved through the head's page table)
 //   warp 1      MMA issuer (one thread): for key tile j, per query tile t,
 //               O_t += P_t(j-1) V(j-1) then S_t(j) = Q_t K(j)^T, all into TMEM
-//   warps 2..5  softmax of query tile 0, warps 6..9 softmax of query tile 1: one thread per
+//   warps 2, 3  idle (they hand their registers to the softmax warpgroups)
+//   warps 4..7  softmax of query tile 0, warps 8..11 softmax of query tile 1: one thread per
 //               row; fp32 online softmax in the exp2 domain, O rescaled only when the row
 //               maximum grows by more than 2^8; P (bf16) overwrites its S columns in TMEM;
 //               the epilogue normalises O and writes bf16 out, fp32 lse and visited counts.
@@ -31,7 +33,11 @@ namespace {
 constexpr int kTileRows = 128;  // rows of one query tile (one TMEM accumulator)
 constexpr int kBN = 128;        // keys of one key tile
 constexpr int kStages = 2;      // K and V ring depth
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Registers per thread: 168 at launch (65536 / 384, and 3 warps x 168 x 32 fit one SM
+// sub-partition's 16384); warpgroup 0 drops to 72 and the two softmax warpgroups rise to
+// 216, which adds up to the launch total: 128 x 72 + 256 x 216 = 384 x 168.
+constexpr int kRegsLow = 72, kRegsHigh = 216;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
 
 template <int D>
@@ -88,8 +94,304 @@ __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const Prefil
   return it;
 }
 
+// ---------------------------------------------------------------------------- producer warp
 template <int D>
-__global__ void __maxnreg__(200)
+__device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUtensorMap &kmap,
+                                              const CUtensorMap &vmap, const PrefillLaunch &p, Bars *bar,
+                                              const PrefillSeq *seqs, const int2 *items, uint8_t *q_s, uint8_t *k_s,
+                                              uint8_t *v_s, int *sched_next, int lane, int G, int32_t *state,
+                                              volatile int *abort_flag) {
+  using S = Smem<D>;
+  if (lane == 0) {
+    tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+  }
+  const int P = p.g.page, PPT = kBN / P;
+  int i = 0, c = 0;
+  bool ok = true, q_loaded = false;
+  for (;;) {
+    int idx = 0;
+    if (lane == 0) idx = atomicAdd(sched_next, 1);
+    idx = __shfl_sync(0xffffffffu, idx, 0);
+    if (idx >= p.n_items) idx = -1;
+    const int slot = i & 3;
+    if (!(ok = warp_wait(&bar->sched_empty[slot], ((i >> 2) & 1) ^ 1, abort_flag, state))) break;
+    if (lane == 0) {
+      bar->sched[slot] = idx;
+      mbar_arrive(&bar->sched_full[slot]);
+    }
+    if (idx < 0) break;
+    const Item it = decode_item(p, seqs, items, idx);
+    if (!(ok = warp_wait(&bar->q_empty, (i & 1) ^ 1, abort_flag, state))) break;
+    if (lane == 0) {
+      mbar_expect_tx(&bar->q_full, 2 * S::kQTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int hh = 0; hh < S::kHalves; ++hh)
+          tma_load_3d(q_s + t * S::kQTileBytes + hh * kTileRows * 128, &qmap, &bar->q_full, hh * 64, it.h * G,
+                      it.q_row + t * p.tile_pos);
+    }
+    q_loaded = true;
+    const long long row_base = (((long long)p.layer * p.g.max_seqs + it.seq_id) * p.g.hkv + it.h) * p.g.max_lp;
+    const int last_lp = (it.kv_len - 1) / P;
+    int lp_base = -(1 << 30), pid = p.g.num_pages;
+    for (int kt = it.kt_lo; kt <= it.kt_hi; ++kt) {
+      const int lp_first = kt * PPT;
+      if (lp_first < lp_base || lp_first + PPT > lp_base + 32) {
+        // resolve 32 logical pages at once, one per lane; pages not stored load zeros
+        lp_base = lp_first;
+        const int lp = lp_base + lane;
+        pid = p.g.num_pages;
+        const bool stored = lp <= last_lp && (it.global || lp >= last_lp - p.g.ring + 1);
+        if (stored) {
+          const int32_t v = p.g.page_table[row_base + (it.global ? lp : lp % p.g.ring)];
+          if (v >= 0 && v < p.g.num_pages) pid = v;
+          else if ((long long)lp * P + P - 1 >= it.lo_min && lp * P <= it.q_last) set_error(state, kErrDeviceBounds);
+        }
+      }
+      const int s = c % kStages;
+      const uint32_t u = (uint32_t)(c / kStages);
+      if (!(ok = warp_wait(&bar->k_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
+      if (lane == 0) mbar_expect_tx(&bar->k_full[s], S::kTileBytes);
+      for (int j = 0; j < PPT; ++j) {
+        const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
+        if (lane == 0)
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            tma_load_3d(k_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, &kmap, &bar->k_full[s], hh * 64, 0,
+                        phys);
+      }
+      if (!(ok = warp_wait(&bar->v_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
+      if (lane == 0) mbar_expect_tx(&bar->v_full[s], S::kTileBytes);
+      for (int j = 0; j < PPT; ++j) {
+        const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
+        if (lane == 0)
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            tma_load_3d(v_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, &vmap, &bar->v_full[s], hh * 64, 0,
+                        phys);
+      }
+      ++c;
+    }
+    if (!ok) break;
+    ++i;
+  }
+  // drain: no copy of this CTA may still be in flight when it exits
+  for (int k = c - 1; k >= 0 && k >= c - kStages; --k) {
+    const int s = k % kStages;
+    const uint32_t u = (uint32_t)(k / kStages);
+    mbar_wait_drain(&bar->k_full[s], u & 1);
+    mbar_wait_drain(&bar->v_full[s], u & 1);
+  }
+  if (q_loaded) mbar_wait_drain(&bar->q_full, (uint32_t)((ok ? i - 1 : i) & 1));
+}
+
+// ---------------------------------------------------------------------------- MMA thread
+template <int D>
+__device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, const PrefillSeq *seqs, const int2 *items,
+                                         uint8_t *q_s, uint8_t *k_s, uint8_t *v_s, uint32_t tmem, int32_t *state,
+                                         volatile int *abort_flag) {
+  using S = Smem<D>;
+  constexpr uint32_t kIdescQK = idesc_bf16(kTileRows, kBN, 0, 0);
+  constexpr uint32_t kIdescPV = idesc_bf16(kTileRows, D, 0, 1);
+  const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
+  int i = 0, c = 0;
+  bool ok = true;
+  // O_t += P_t(cc) V(cc); the first PV of an item overwrites O_t
+  auto issue_pv = [&](int t, int cc, bool first) -> bool {
+    const int s = cc % kStages;
+    if (!mbar_wait(&bar->p_ready[t], cc & 1, abort_flag, state)) return false;
+    if (t == 0 && !mbar_wait(&bar->v_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
+    if (first && !mbar_wait(&bar->o_free[t], (i & 1) ^ 1, abort_flag, state)) return false;
+    tc_fence_after();
+    const uint32_t vb = v_addr + s * S::kTileBytes;
+#pragma unroll
+    for (int kk = 0; kk < kBN / 16; ++kk)
+      umma_ts(tmem + S::col_o(t), tmem + S::col_s(t) + kk * 8, sdesc_sw128(vb + kk * 2048, kBN * 128, 1024),
+              kIdescPV, (!first || kk > 0) ? 1u : 0u);
+    umma_commit(&bar->pv_done[t]);
+    return true;
+  };
+  // S_t(cc) = Q_t K(cc)^T
+  auto issue_s = [&](int t, int cc) {
+    const uint32_t kb = k_addr + (cc % kStages) * S::kTileBytes;
+    const uint32_t qb = q_addr + t * S::kQTileBytes;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off_q = (kk >> 2) * (kTileRows * 128) + (kk & 3) * 32;
+      const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+      umma_ss(tmem + S::col_s(t), sdesc_sw128(qb + off_q, 16, 1024), sdesc_sw128(kb + off_k, 16, 1024),
+              kIdescQK, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&bar->s_full[t]);
+  };
+  for (;;) {
+    const int slot = i & 3;
+    if (!(ok = mbar_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state))) break;
+    const int idx = bar->sched[slot];
+    mbar_arrive(&bar->sched_empty[slot]);
+    if (idx < 0) break;
+    const Item it = decode_item(p, seqs, items, idx);
+    const int n_tiles = it.kt_hi - it.kt_lo + 1;
+    if (!(ok = mbar_wait(&bar->q_full, i & 1, abort_flag, state))) break;
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      const int s = c % kStages;
+      if (!(ok = mbar_wait(&bar->k_full[s], (uint32_t)(c / kStages) & 1, abort_flag, state))) break;
+      tc_fence_after();
+      for (int t = 0; t < 2; ++t) {
+        if (j > 0 && !(ok = issue_pv(t, c - 1, j == 1))) break;
+        issue_s(t, c);
+      }
+      if (!ok) break;
+      umma_commit(&bar->k_empty[s]);
+      if (j > 0) umma_commit(&bar->v_empty[(c - 1) % kStages]);
+      if (j == n_tiles - 1) umma_commit(&bar->q_empty);
+      ++c;
+    }
+    if (!ok) break;
+    for (int t = 0; t < 2 && ok; ++t) ok = issue_pv(t, c - 1, n_tiles == 1);
+    if (!ok) break;
+    umma_commit(&bar->v_empty[(c - 1) % kStages]);
+    ++i;
+  }
+  // every MMA issued by this thread must finish before TMEM is released
+  umma_commit(&bar->mma_done);
+  mbar_wait_drain(&bar->mma_done, 0);
+}
+
+// ---------------------------------------------------------------------------- softmax warpgroups
+template <int D>
+__device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, const PrefillSeq *seqs,
+                                             const int2 *items, uint32_t tmem, int warp, int lane, int G,
+                                             int32_t *state, volatile int *abort_flag) {
+  using S = Smem<D>;
+  const int tq = (warp - 4) >> 2;  // query tile of this warpgroup
+  const int q4 = warp & 3;         // TMEM lane quadrant of this warp
+  const int row = q4 * 32 + lane;
+  const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
+  const uint32_t t_s = t_lane + S::col_s(tq), t_o = t_lane + S::col_o(tq);
+  const float sl2 = p.scale_log2;
+  int i = 0, c = 0;
+  for (;;) {
+    const int slot = i & 3;
+    if (!warp_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state)) break;
+    const int idx = bar->sched[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar->sched_empty[slot]);
+    if (idx < 0) break;
+    const Item it = decode_item(p, seqs, items, idx);
+    const int n_tiles = it.kt_hi - it.kt_lo + 1;
+    const int pos_local = tq * p.tile_pos + row / G, g = row % G;
+    const int p_raw = it.q_first + pos_local;
+    const bool valid = p_raw <= it.q_last;
+    const int pq = min(p_raw, it.q_last);  // rows past the sequence repeat its last query
+    const int lo = it.global ? 0 : max(0, pq - p.g.window + 1);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      if (!(ok = warp_wait(&bar->s_full[tq], c & 1, abort_flag, state))) break;
+      tc_fence_after();
+      float s[kBN];
+#pragma unroll
+      for (int cc = 0; cc < kBN / 16; ++cc)
+        tmem_ld16(t_s + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[cc * 16]));
+      tmem_ld_wait();
+      const int k0 = (it.kt_lo + j) * kBN;
+      if (k0 < lo || k0 + kBN - 1 > pq) {
+#pragma unroll
+        for (int jj = 0; jj < kBN; ++jj) {
+          const int kp = k0 + jj;
+          if (kp < lo || kp > pq) s[jj] = -INFINITY;
+        }
+      }
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+#pragma unroll
+      for (int jj = 8; jj < kBN; jj += 8)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], s[jj + e]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_new = mx * sl2;  // -inf stays -inf (scale > 0)
+      const bool grow = m_new > m_used + kRescaleThreshold;
+      // O_t holds earlier tiles' sums scaled by m_used.  The PV that last wrote it has
+      // completed: it was issued before this tile's S, whose completion we waited for.
+      // TMEM loads/stores need the whole warp, so the warp rescales when any row must,
+      // with factor 1 for the others.
+      const bool rescale = grow && m_used != -INFINITY;
+      if (__any_sync(0xffffffffu, rescale)) {
+        const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.0f;
+#pragma unroll
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t o[16];
+          tmem_ld16(t_o + cc * 16, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(t_o + cc * 16, o);
+        }
+        l *= alpha;
+      }
+      if (grow) m_used = m_new;
+      // P = exp2(s * scale_log2 - m_used), written as bf16 pairs over the S columns
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int cc = 0; cc < kBN / 32; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a = fast_exp2(fmaf(s[cc * 32 + 2 * e], sl2, neg_m));
+          const float b2 = fast_exp2(fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m));
+          rs[e & 3] += a + b2;
+          pk[e] = pack_bf16x2(a, b2);
+        }
+        tmem_st16(t_s + cc * 16, pk);
+      }
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bar->p_ready[tq]);
+      ++c;
+    }
+    if (!ok) break;
+    // epilogue: the item's last PV into O_t
+    if (!warp_wait(&bar->pv_done[tq], (c - 1) & 1, abort_flag, state)) break;
+    tc_fence_after();
+    const float inv_l = (valid && l > 0.f) ? 1.f / l : 0.f;
+    const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
+#pragma unroll
+    for (int cc = 0; cc < D / 16; ++cc) {
+      uint32_t o[16];
+      tmem_ld16(t_o + cc * 16, o);
+      tmem_ld_wait();
+      uint32_t w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+      if (valid) {
+        dst[cc * 2 + 0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[cc * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(&bar->o_free[tq]);
+    if (valid) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;
+    if (p.visited) {
+      unsigned long long cnt = valid ? (unsigned long long)(pq - lo + 1) : 0ull;
+      if (G < 32) {
+        for (int off = G; off < 32; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+        if (lane < G && cnt) atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + lane], cnt);
+      } else if (cnt) {
+        atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + g], cnt);
+      }
+    }
+    ++i;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const PrefillLaunch p) {
   using S = Smem<D>;
@@ -138,283 +440,15 @@ __global__ void __maxnreg__(200)
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&qmap);
-      tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
-    }
-    const int P = p.g.page, PPT = kBN / P;
-    int i = 0, c = 0;
-    bool ok = true, q_loaded = false;
-    for (;;) {
-      int idx = 0;
-      if (lane == 0) idx = atomicAdd(sched_next, 1);
-      idx = __shfl_sync(0xffffffffu, idx, 0);
-      if (idx >= p.n_items) idx = -1;
-      const int slot = i & 3;
-      if (!(ok = warp_wait(&bar->sched_empty[slot], ((i >> 2) & 1) ^ 1, abort_flag, state))) break;
-      if (lane == 0) {
-        bar->sched[slot] = idx;
-        mbar_arrive(&bar->sched_full[slot]);
-      }
-      if (idx < 0) break;
-      const Item it = decode_item(p, seqs, items, idx);
-      if (!(ok = warp_wait(&bar->q_empty, (i & 1) ^ 1, abort_flag, state))) break;
-      if (lane == 0) {
-        mbar_expect_tx(&bar->q_full, 2 * S::kQTileBytes);
-        for (int t = 0; t < 2; ++t)
-          for (int hh = 0; hh < S::kHalves; ++hh)
-            tma_load_3d(q_s + t * S::kQTileBytes + hh * kTileRows * 128, &qmap, &bar->q_full, hh * 64, it.h * G,
-                        it.q_row + t * p.tile_pos);
-      }
-      q_loaded = true;
-      const long long row_base = (((long long)p.layer * p.g.max_seqs + it.seq_id) * p.g.hkv + it.h) * p.g.max_lp;
-      const int last_lp = (it.kv_len - 1) / P;
-      int lp_base = -(1 << 30), pid = p.g.num_pages;
-      for (int kt = it.kt_lo; kt <= it.kt_hi; ++kt) {
-        const int lp_first = kt * PPT;
-        if (lp_first < lp_base || lp_first + PPT > lp_base + 32) {
-          // resolve 32 logical pages at once, one per lane; pages not stored load zeros
-          lp_base = lp_first;
-          const int lp = lp_base + lane;
-          pid = p.g.num_pages;
-          const bool stored = lp <= last_lp && (it.global || lp >= last_lp - p.g.ring + 1);
-          if (stored) {
-            const int32_t v = p.g.page_table[row_base + (it.global ? lp : lp % p.g.ring)];
-            if (v >= 0 && v < p.g.num_pages) pid = v;
-            else if ((long long)lp * P + P - 1 >= it.lo_min && lp * P <= it.q_last) set_error(state, kErrDeviceBounds);
-          }
-        }
-        const int s = c % kStages;
-        const uint32_t u = (uint32_t)(c / kStages);
-        if (!(ok = warp_wait(&bar->k_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
-        if (lane == 0) mbar_expect_tx(&bar->k_full[s], S::kTileBytes);
-        for (int j = 0; j < PPT; ++j) {
-          const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
-          if (lane == 0)
-            for (int hh = 0; hh < S::kHalves; ++hh)
-              tma_load_3d(k_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, &kmap, &bar->k_full[s], hh * 64, 0,
-                          phys);
-        }
-        if (!(ok = warp_wait(&bar->v_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
-        if (lane == 0) mbar_expect_tx(&bar->v_full[s], S::kTileBytes);
-        for (int j = 0; j < PPT; ++j) {
-          const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
-          if (lane == 0)
-            for (int hh = 0; hh < S::kHalves; ++hh)
-              tma_load_3d(v_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, &vmap, &bar->v_full[s], hh * 64, 0,
-                          phys);
-        }
-        ++c;
-      }
-      if (!ok) break;
-      ++i;
-    }
-    // drain: no copy of this CTA may still be in flight when it exits
-    for (int k = c - 1; k >= 0 && k >= c - kStages; --k) {
-      const int s = k % kStages;
-      const uint32_t u = (uint32_t)(k / kStages);
-      mbar_wait_drain(&bar->k_full[s], u & 1);
-      mbar_wait_drain(&bar->v_full[s], u & 1);
-    }
-    if (q_loaded) mbar_wait_drain(&bar->q_full, (uint32_t)((ok ? i - 1 : i) & 1));
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdescQK = idesc_bf16(kTileRows, kBN, 0, 0);
-      constexpr uint32_t kIdescPV = idesc_bf16(kTileRows, D, 0, 1);
-      const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
-      int i = 0, c = 0;
-      bool ok = true;
-      // O_t += P_t(cc) V(cc); the first PV of an item overwrites O_t
-      auto issue_pv = [&](int t, int cc, bool first) -> bool {
-        const int s = cc % kStages;
-        if (!mbar_wait(&bar->p_ready[t], cc & 1, abort_flag, state)) return false;
-        if (t == 0 && !mbar_wait(&bar->v_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
-        if (first && !mbar_wait(&bar->o_free[t], (i & 1) ^ 1, abort_flag, state)) return false;
-        tc_fence_after();
-        const uint32_t vb = v_addr + s * S::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tmem + S::col_o(t), tmem + S::col_s(t) + kk * 8, sdesc_sw128(vb + kk * 2048, kBN * 128, 1024),
-                  kIdescPV, (!first || kk > 0) ? 1u : 0u);
-        umma_commit(&bar->pv_done[t]);
-        return true;
-      };
-      // S_t(cc) = Q_t K(cc)^T
-      auto issue_s = [&](int t, int cc) {
-        const uint32_t kb = k_addr + (cc % kStages) * S::kTileBytes;
-        const uint32_t qb = q_addr + t * S::kQTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_q = (kk >> 2) * (kTileRows * 128) + (kk & 3) * 32;
-          const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          umma_ss(tmem + S::col_s(t), sdesc_sw128(qb + off_q, 16, 1024), sdesc_sw128(kb + off_k, 16, 1024),
-                  kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&bar->s_full[t]);
-      };
-      for (;;) {
-        const int slot = i & 3;
-        if (!(ok = mbar_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state))) break;
-        const int idx = bar->sched[slot];
-        mbar_arrive(&bar->sched_empty[slot]);
-        if (idx < 0) break;
-        const Item it = decode_item(p, seqs, items, idx);
-        const int n_tiles = it.kt_hi - it.kt_lo + 1;
-        if (!(ok = mbar_wait(&bar->q_full, i & 1, abort_flag, state))) break;
-        for (int j = 0; j < n_tiles && ok; ++j) {
-          const int s = c % kStages;
-          if (!(ok = mbar_wait(&bar->k_full[s], (uint32_t)(c / kStages) & 1, abort_flag, state))) break;
-          tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (j > 0 && !(ok = issue_pv(t, c - 1, j == 1))) break;
-            issue_s(t, c);
-          }
-          if (!ok) break;
-          umma_commit(&bar->k_empty[s]);
-          if (j > 0) umma_commit(&bar->v_empty[(c - 1) % kStages]);
-          if (j == n_tiles - 1) umma_commit(&bar->q_empty);
-          ++c;
-        }
-        if (!ok) break;
-        for (int t = 0; t < 2 && ok; ++t) ok = issue_pv(t, c - 1, n_tiles == 1);
-        if (!ok) break;
-        umma_commit(&bar->v_empty[(c - 1) % kStages]);
-        ++i;
-      }
-      // every MMA issued by this thread must finish before TMEM is released
-      umma_commit(&bar->mma_done);
-      mbar_wait_drain(&bar->mma_done, 0);
-    }
+  if (warp >= 4) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+    softmax_role<D>(p, bar, seqs, items, tmem, warp, lane, G, state, abort_flag);
   } else {
-    // ------------------------------------------------------------------ softmax / epilogue
-    const int tq = (warp - 2) >> 2;  // query tile of this warpgroup
-    const int q4 = warp & 3;         // TMEM lane quadrant of this warp
-    const int row = q4 * 32 + lane;
-    const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
-    const uint32_t t_s = t_lane + S::col_s(tq), t_o = t_lane + S::col_o(tq);
-    const float sl2 = p.scale_log2;
-    int i = 0, c = 0;
-    for (;;) {
-      const int slot = i & 3;
-      if (!warp_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state)) break;
-      const int idx = bar->sched[slot];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->sched_empty[slot]);
-      if (idx < 0) break;
-      const Item it = decode_item(p, seqs, items, idx);
-      const int n_tiles = it.kt_hi - it.kt_lo + 1;
-      const int pos_local = tq * p.tile_pos + row / G, g = row % G;
-      const int p_raw = it.q_first + pos_local;
-      const bool valid = p_raw <= it.q_last;
-      const int pq = min(p_raw, it.q_last);  // rows past the sequence repeat its last query
-      const int lo = it.global ? 0 : max(0, pq - p.g.window + 1);
-      float m_used = -INFINITY, l = 0.f;
-      bool ok = true;
-      for (int j = 0; j < n_tiles; ++j) {
-        if (!(ok = warp_wait(&bar->s_full[tq], c & 1, abort_flag, state))) break;
-        tc_fence_after();
-        float s[kBN];
-#pragma unroll
-        for (int cc = 0; cc < kBN / 16; ++cc)
-          tmem_ld16(t_s + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[cc * 16]));
-        tmem_ld_wait();
-        const int k0 = (it.kt_lo + j) * kBN;
-        if (k0 < lo || k0 + kBN - 1 > pq) {
-#pragma unroll
-          for (int jj = 0; jj < kBN; ++jj) {
-            const int kp = k0 + jj;
-            if (kp < lo || kp > pq) s[jj] = -INFINITY;
-          }
-        }
-        float mx8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = s[e];
-#pragma unroll
-        for (int jj = 8; jj < kBN; jj += 8)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], s[jj + e]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float m_new = mx * sl2;  // -inf stays -inf (scale > 0)
-        const bool grow = m_new > m_used + kRescaleThreshold;
-        // O_t holds earlier tiles' sums scaled by m_used.  The PV that last wrote it has
-        // completed: it was issued before this tile's S, whose completion we waited for.
-        // TMEM loads/stores need the whole warp, so the warp rescales when any row must,
-        // with factor 1 for the others.
-        const bool rescale = grow && m_used != -INFINITY;
-        if (__any_sync(0xffffffffu, rescale)) {
-          const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.0f;
-#pragma unroll
-          for (int cc = 0; cc < D / 16; ++cc) {
-            uint32_t o[16];
-            tmem_ld16(t_o + cc * 16, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16(t_o + cc * 16, o);
-          }
-          l *= alpha;
-        }
-        if (grow) m_used = m_new;
-        // P = exp2(s * scale_log2 - m_used), written as bf16 pairs over the S columns
-        const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float a = fast_exp2(fmaf(s[cc * 32 + 2 * e], sl2, neg_m));
-            const float b2 = fast_exp2(fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m));
-            rs[e & 3] += a + b2;
-            pk[e] = pack_bf16x2(a, b2);
-          }
-          tmem_st16(t_s + cc * 16, pk);
-        }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bar->p_ready[tq]);
-        ++c;
-      }
-      if (!ok) break;
-      // epilogue: the item's last PV into O_t
-      if (!warp_wait(&bar->pv_done[tq], (c - 1) & 1, abort_flag, state)) break;
-      tc_fence_after();
-      const float inv_l = (valid && l > 0.f) ? 1.f / l : 0.f;
-      const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
-#pragma unroll
-      for (int cc = 0; cc < D / 16; ++cc) {
-        uint32_t o[16];
-        tmem_ld16(t_o + cc * 16, o);
-        tmem_ld_wait();
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (valid) {
-          dst[cc * 2 + 0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[cc * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bar->o_free[tq]);
-      if (valid) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;
-      if (p.visited) {
-        unsigned long long cnt = valid ? (unsigned long long)(pq - lo + 1) : 0ull;
-        if (G < 32) {
-          for (int off = G; off < 32; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-          if (lane < G && cnt) atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + lane], cnt);
-        } else if (cnt) {
-          atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + g], cnt);
-        }
-      }
-      ++i;
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    if (warp == 0) {
+      producer_role<D>(qmap, kmap, vmap, p, bar, seqs, items, q_s, k_s, v_s, sched_next, lane, G, state, abort_flag);
+    } else if (warp == 1 && lane == 0) {
+      mma_role<D>(p, bar, seqs, items, q_s, k_s, v_s, tmem, state, abort_flag);
     }
   }
 

@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstring>
 #include <new>
+#include <string>
 #include <vector>
 
 #include "../../include/segkv.h"
@@ -78,9 +79,20 @@ struct segkv {
   bool maps_ready = false;
   CUtensorMap kmap, vmap;
   int num_sms = 0;
+  std::string last_error;  // which CUDA step failed last, and why
 };
 
 namespace {
+
+int cuda_fail(segkv_t *h, const char *what, cudaError_t e) {
+  h->last_error = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return SEGKV_ERR_CUDA;
+}
+#define SEGKV_CUDA(h, what, expr)                    \
+  do {                                               \
+    const cudaError_t e_ = (expr);                   \
+    if (e_ != cudaSuccess) return cuda_fail(h, what, e_); \
+  } while (0)
 
 StorageGeom geom(const segkv_t *h) {
   StorageGeom g;
@@ -111,16 +123,16 @@ int held_pages(const segkv_t *h, bool global, int n) {
 int staging(segkv_t *h, size_t bytes, void **host) {
   Staging &s = h->slot[h->next_slot];
   if (s.pending) {
-    if (cudaEventSynchronize(s.ev) != cudaSuccess) return SEGKV_ERR_CUDA;
+    SEGKV_CUDA(h, "staging event wait", cudaEventSynchronize(s.ev));
     s.pending = false;
   }
-  if (!s.ev && cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming) != cudaSuccess) return SEGKV_ERR_CUDA;
+  if (!s.ev) SEGKV_CUDA(h, "staging event create", cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming));
   if (s.cap < bytes) {
     if (s.host) cudaFreeHost(s.host);
     s.host = nullptr;
     s.cap = 0;
     const size_t cap = std::max<size_t>(align_up(bytes, 4096), 64 << 10);
-    if (cudaHostAlloc(&s.host, cap, cudaHostAllocDefault) != cudaSuccess) return SEGKV_ERR_CUDA;
+    SEGKV_CUDA(h, "pinned staging alloc", cudaHostAlloc(&s.host, cap, cudaHostAllocDefault));
     s.cap = cap;
   }
   *host = s.host;
@@ -129,8 +141,8 @@ int staging(segkv_t *h, size_t bytes, void **host) {
 
 int upload(segkv_t *h, void *ws, size_t bytes, cudaStream_t st) {
   Staging &s = h->slot[h->next_slot];
-  if (cudaMemcpyAsync(ws, s.host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return SEGKV_ERR_CUDA;
-  if (cudaEventRecord(s.ev, st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  SEGKV_CUDA(h, "metadata upload", cudaMemcpyAsync(ws, s.host, bytes, cudaMemcpyHostToDevice, st));
+  SEGKV_CUDA(h, "staging event record", cudaEventRecord(s.ev, st));
   s.pending = true;
   h->next_slot = (h->next_slot + 1) % kStagingSlots;
   return SEGKV_OK;
@@ -139,13 +151,15 @@ int upload(segkv_t *h, void *ws, size_t bytes, cudaStream_t st) {
 int ensure_device_state(segkv_t *h) {
   if (h->maps_ready) return SEGKV_OK;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SEGKV_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SEGKV_ERR_CUDA;
+  SEGKV_CUDA(h, "cudaGetDevice", cudaGetDevice(&dev));
+  SEGKV_CUDA(h, "SM count", cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
   const segkv_config &c = h->cfg;
   const uint64_t rowb = (uint64_t)c.head_dim * 2, pageb = rowb * c.page_size;
   if (!make_map(&h->kmap, c.k_pool, c.head_dim, c.page_size, c.num_pages, rowb, pageb, c.page_size, 1) ||
-      !make_map(&h->vmap, c.v_pool, c.head_dim, c.page_size, c.num_pages, rowb, pageb, c.page_size, 1))
+      !make_map(&h->vmap, c.v_pool, c.head_dim, c.page_size, c.num_pages, rowb, pageb, c.page_size, 1)) {
+    h->last_error = "pool tensor map encode failed";
     return SEGKV_ERR_CUDA;
+  }
   h->maps_ready = true;
   return SEGKV_OK;
 }
@@ -278,6 +292,7 @@ void segkv_destroy(segkv_t *h) {
 }
 
 int segkv_ring_pages(const segkv_t *h) { return h ? h->ring : -1; }
+const char *segkv_last_error(const segkv_t *h) { return h ? h->last_error.c_str() : "no handle"; }
 int segkv_max_lp(const segkv_t *h) { return h ? h->max_lp : -1; }
 int segkv_pages_used(const segkv_t *h) { return h ? (int)h->pages_used : -1; }
 
@@ -303,8 +318,7 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
 
 int segkv_reset(segkv_t *h, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
-  if (launch_reset(geom(h), h->cfg.num_layers, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return SEGKV_ERR_CUDA;
+  SEGKV_CUDA(h, "reset launch", launch_reset(geom(h), h->cfg.num_layers, static_cast<cudaStream_t>(stream)));
   std::fill(h->len.begin(), h->len.end(), 0);
   h->pages_used = 0;
   return SEGKV_OK;
@@ -351,8 +365,7 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = upload(h, ws, bytes, st))) return rc;
   const uint8_t *cls_dev = static_cast<const uint8_t *>(ws) + kHeaderBytes + sizeof(AppendSeq) * nseq;
-  if (launch_append(geom(h), layer, ws, nseq, cls_dev, (int)total, k_new, v_new, st) != cudaSuccess)
-    return SEGKV_ERR_CUDA;
+  SEGKV_CUDA(h, "append launch", launch_append(geom(h), layer, ws, nseq, cls_dev, (int)total, k_new, v_new, st));
   for (int b = 0; b < nseq; ++b) h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] += num_new[b];
   h->pages_used += new_pages;
   return SEGKV_OK;
@@ -419,8 +432,11 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
     it[i] = make_int2(items[i].b, (int)make_item_w1(h->cls[layer * H + items[i].h] != 0, items[i].h, items[i].t));
   CUtensorMap qmap;
   const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads;
-  if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G, kPrefillTileRows / h->G))
+  if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
+                kPrefillTileRows / h->G)) {
+    h->last_error = "query tensor map encode failed";
     return SEGKV_ERR_CUDA;
+  }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = upload(h, ws, bytes, st))) return rc;
   PrefillLaunch p;
@@ -438,7 +454,7 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
   p.visited = reinterpret_cast<unsigned long long *>(visited);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
-  if (launch_prefill(p, qmap, h->kmap, h->vmap, st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  SEGKV_CUDA(h, "prefill launch", launch_prefill(p, qmap, h->kmap, h->vmap, st));
   return SEGKV_OK;
 }
 
@@ -526,7 +542,7 @@ int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
   p.visited = reinterpret_cast<unsigned long long *>(visited);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
-  if (launch_decode(p, h->kmap, h->vmap, st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  SEGKV_CUDA(h, "decode launch", launch_decode(p, h->kmap, h->vmap, st));
   return SEGKV_OK;
 }
 
@@ -534,11 +550,10 @@ int segkv_device_status(segkv_t *h, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t word = 0;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return SEGKV_ERR_CUDA;
-  if (cudaMemcpyAsync(&word, h->cfg.state + 1, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return SEGKV_ERR_CUDA;
-  if (cudaMemsetAsync(h->cfg.state + 1, 0, sizeof(int32_t), st) != cudaSuccess) return SEGKV_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return SEGKV_ERR_CUDA;
+  SEGKV_CUDA(h, "status sync", cudaStreamSynchronize(st));
+  SEGKV_CUDA(h, "status read", cudaMemcpyAsync(&word, h->cfg.state + 1, sizeof(word), cudaMemcpyDeviceToHost, st));
+  SEGKV_CUDA(h, "status clear", cudaMemsetAsync(h->cfg.state + 1, 0, sizeof(int32_t), st));
+  SEGKV_CUDA(h, "status sync", cudaStreamSynchronize(st));
   return word;
 }
 

@@ -24,7 +24,7 @@ STATUS = {
 EXPORTS = [
     "segkv_create", "segkv_destroy", "segkv_ring_pages", "segkv_max_lp", "segkv_seq_len", "segkv_pages_used",
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
-    "segkv_decode_attn", "segkv_device_status", "segkv_strerror",
+    "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
 ]
 
 
@@ -72,15 +72,20 @@ def lib():
                                          ctypes.POINTER(I)]
         L.segkv_decode_attn.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P, SZ, P]
         L.segkv_device_status.argtypes = [P, P]
+        L.segkv_last_error.argtypes = [P]
+        L.segkv_last_error.restype = ctypes.c_char_p
         L.segkv_strerror.argtypes = [I]
         L.segkv_strerror.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
 
-def _check(rc: int, what: str) -> None:
+def _check(rc: int, what: str, h=None) -> None:
     if rc != SEGKV_OK:
-        raise SegkvError(rc, what)
+        detail = ""
+        if h is not None and rc == 6:
+            detail = " [" + lib().segkv_last_error(h).decode(errors="replace") + "]"
+        raise SegkvError(rc, what + detail)
 
 
 def _i32(x) -> np.ndarray:
@@ -150,7 +155,7 @@ class Handle:
         return lib().segkv_workspace_bytes(self.h, max_batch, max_tokens)
 
     def reset(self, stream=None) -> None:
-        _check(lib().segkv_reset(self.h, _stream(stream)), "segkv_reset")
+        _check(lib().segkv_reset(self.h, _stream(stream)), "segkv_reset", self.h)
 
     def append(self, layer, seq_ids, start, count, k_new, v_new, ws, ws_bytes, stream=None) -> int:
         s, st, c = _i32(seq_ids), _i32(start), _i32(count)
@@ -228,7 +233,7 @@ class SegKV:
 
     def append(self, layer: int, seq_ids: Sequence[int], start: Sequence[int], count: Sequence[int], k_new, v_new):
         _check(self.handle.append(layer, seq_ids, start, count, k_new, v_new, self.ws, self.ws_bytes),
-               "segkv_append")
+               "segkv_append", self.handle.h)
 
     def prefill(self, layer: int, seq_ids, q_start, q_len, q, *, out=None, lse=None, visited=None,
                 scale: float = 0.0):
@@ -237,7 +242,7 @@ class SegKV:
         out = out if out is not None else t.empty((T, self.hq, self.d), dtype=t.bfloat16, device=self.device)
         lse = lse if lse is not None else t.empty((T, self.hq), dtype=t.float32, device=self.device)
         _check(self.handle.prefill(layer, seq_ids, q_start, q_len, q, scale, out, lse, visited, self.ws,
-                                   self.ws_bytes), "segkv_prefill_attn")
+                                   self.ws_bytes), "segkv_prefill_attn", self.handle.h)
         return out, lse
 
     def decode(self, layer: int, seq_ids, q_pos, q, *, out=None, lse=None, visited=None, scale: float = 0.0,
@@ -247,7 +252,7 @@ class SegKV:
         out = out if out is not None else t.empty((B, self.hq, self.d), dtype=t.bfloat16, device=self.device)
         lse = lse if lse is not None else t.empty((B, self.hq), dtype=t.float32, device=self.device)
         _check(self.handle.decode(layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, self.ws,
-                                  self.ws_bytes), "segkv_decode_attn")
+                                  self.ws_bytes), "segkv_decode_attn", self.handle.h)
         return out, lse
 
     def device_status(self) -> int:

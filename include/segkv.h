@@ -164,6 +164,10 @@ int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
  * (SEGKV_OK, SEGKV_ERR_DEVICE_BOUNDS or SEGKV_ERR_DEVICE_TIMEOUT), or SEGKV_ERR_CUDA. */
 int segkv_device_status(segkv_t *h, void *stream);
 
+/* What the last SEGKV_ERR_CUDA of this handle came from (the failing step and the CUDA
+ * error name), or "" if none.  The string belongs to the handle. */
+const char *segkv_last_error(const segkv_t *h);
+
 /* Static description of a status code. */
 const char *segkv_strerror(int status);
 

@@ -75,8 +75,8 @@ def closed_form_counts(w, layer, ids, qs, ql):
 
 def prefill_full(torch, w, layer_list, n_rows, ctx_chunk=4096, golden=None):
     kv = make_kv(w)
+    o = orc.Oracle.for_workload(w)  # one allocator for all layers, like the library's
     for layer in layer_list:
-        o = orc.Oracle.for_workload(w)
         dual_replay(w, layer, kv, o, ctx_chunk)
         ids, qs, ql = step_queries(w)
         q = q_for_call(w, layer, ids, qs, ql)
@@ -94,7 +94,7 @@ def prefill_full(torch, w, layer_list, n_rows, ctx_chunk=4096, golden=None):
             for h in range(w.hq):
                 assert int(got[0, h]) == (g["global"] if w.classes[layer][h // w.group] else g["local"])
         assert np.array_equal(kv.page_table.cpu().numpy()[layer], o.page_table()[layer])
-        del o
+    assert int(kv.state[0].item()) == o.cursor
     return kv
 
 

@@ -9,21 +9,24 @@
 // Work item = two 128-row query tiles of one (sequence, KV head): each tile packs the G
 // query heads of the KV head over 128/G consecutive positions (GQA group packing), and the
 // two tiles cover 256/G consecutive positions.  Both tiles share every K/V tile load.
+// Key tiles hold BN = 64 keys.  Each query tile owns two S buffers in TMEM, so the tensor
+// core computes S(j+1) while the softmax warps work on S(j).
 //
 // One persistent CTA per SM, 384 threads (three warpgroups; one warp of each per SM
 // sub-partition, so the softmax warps can hold a 128-column S row in registers):
 //   warp 0      producer: takes the next item of the longest-first list (atomic counter),
 //               loads both Q tiles once, then streams K and V tiles page by page through TMA
-//               (a tile of BN = 128 keys is BN/P pages resolved through the head's page table)
-//   warp 1      MMA issuer (one thread): for key tile j, per query tile t,
-//               O_t += P_t(j-1) V(j-1) then S_t(j) = Q_t K(j)^T, all into TMEM
+//               (a tile of BN = 64 keys is BN/P pages resolved through the head's page table)
+//   warp 1      MMA issuer (one thread): for key tile j, S_t(j+1) = Q_t K(j+1)^T for both
+//               query tiles, then O_t += P_t(j) V(j) as each tile's P becomes ready
 //   warps 2, 3  idle (they hand their registers to the softmax warpgroups)
 //   warps 4..7  softmax of query tile 0, warps 8..11 softmax of query tile 1: one thread per
 //               row; fp32 online softmax in the exp2 domain, O rescaled only when the row
 //               maximum grows by more than 2^8; P (bf16) overwrites its S columns in TMEM;
 //               the epilogue normalises O and writes bf16 out, fp32 lse and visited counts.
-// The two query tiles' chains (S -> softmax -> PV -> next S) interleave on the tensor core:
-// while one tile's warpgroup runs its softmax, the other tile's MMAs run.
+// P_t(j) is written as bf16 over the first half of the S buffer it came from; S_t(j+2)
+// reuses that buffer only after PV_t(j) has been issued (tcgen05 ops of one thread run in
+// issue order).
 #include "device_common.cuh"
 
 namespace skv {
@@ -31,8 +34,8 @@ namespace skv {
 namespace {
 
 constexpr int kTileRows = 128;  // rows of one query tile (one TMEM accumulator)
-constexpr int kBN = 128;        // keys of one key tile
-constexpr int kStages = 2;      // K and V ring depth
+constexpr int kBN = 64;         // keys of one key tile
+constexpr int kStages = 4;      // K and V ring depth
 constexpr int kThreads = 384;
 // Registers per thread: 168 at launch (65536 / 384, and 3 warps x 168 x 32 fit one SM
 // sub-partition's 16384); warpgroup 0 drops to 72 and the two softmax warpgroups rise to
@@ -49,15 +52,16 @@ struct Smem {
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   static constexpr int kBytes = 1024 + kBarOff + 512;
-  // TMEM columns: S_t at 128 t, O_t at 256 + 128 t
-  static constexpr uint32_t col_s(int t) { return 128u * t; }
+  // TMEM columns: S buffer b of query tile t at 128 t + 64 b, O_t at 256 + 128 t
+  static constexpr uint32_t col_s(int t, int b) { return 128u * t + 64u * b; }
   static constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
 };
 
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_ready[2], pv_done[2], o_free[2];
+  uint64_t s_full[2][2], p_ready[2][2], pv_done[2][2];  // [query tile][S buffer]
+  uint64_t o_free[2];
   uint64_t mma_done;
   uint64_t sched_full[4], sched_empty[4];
   int sched[4];
@@ -185,6 +189,8 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
 }
 
 // ---------------------------------------------------------------------------- MMA thread
+// Key tile counter c runs over every tile this CTA processes; tile c uses K/V stage
+// c % kStages and S buffer c & 1 of each query tile.
 template <int D>
 __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, const PrefillSeq *seqs, const int2 *items,
                                          uint8_t *q_s, uint8_t *k_s, uint8_t *v_s, uint32_t tmem, int32_t *state,
@@ -195,33 +201,43 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
   const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
   int i = 0, c = 0;
   bool ok = true;
-  // O_t += P_t(cc) V(cc); the first PV of an item overwrites O_t
-  auto issue_pv = [&](int t, int cc, bool first) -> bool {
+  // S_t(cc) = Q_t K(cc)^T for both query tiles, then release K stage
+  auto issue_s = [&](int cc) -> bool {
     const int s = cc % kStages;
-    if (!mbar_wait(&bar->p_ready[t], cc & 1, abort_flag, state)) return false;
-    if (t == 0 && !mbar_wait(&bar->v_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
-    if (first && !mbar_wait(&bar->o_free[t], (i & 1) ^ 1, abort_flag, state)) return false;
+    if (!mbar_wait(&bar->k_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
     tc_fence_after();
-    const uint32_t vb = v_addr + s * S::kTileBytes;
+    const uint32_t kb = k_addr + s * S::kTileBytes;
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t qb = q_addr + t * S::kQTileBytes;
 #pragma unroll
-    for (int kk = 0; kk < kBN / 16; ++kk)
-      umma_ts(tmem + S::col_o(t), tmem + S::col_s(t) + kk * 8, sdesc_sw128(vb + kk * 2048, kBN * 128, 1024),
-              kIdescPV, (!first || kk > 0) ? 1u : 0u);
-    umma_commit(&bar->pv_done[t]);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off_q = (kk >> 2) * (kTileRows * 128) + (kk & 3) * 32;
+        const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+        umma_ss(tmem + S::col_s(t, cc & 1), sdesc_sw128(qb + off_q, 16, 1024), sdesc_sw128(kb + off_k, 16, 1024),
+                kIdescQK, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&bar->s_full[t][cc & 1]);
+    }
+    umma_commit(&bar->k_empty[s]);
     return true;
   };
-  // S_t(cc) = Q_t K(cc)^T
-  auto issue_s = [&](int t, int cc) {
-    const uint32_t kb = k_addr + (cc % kStages) * S::kTileBytes;
-    const uint32_t qb = q_addr + t * S::kQTileBytes;
+  // O_t += P_t(cc) V(cc) for both query tiles (the first tile of an item overwrites O_t)
+  auto issue_pv = [&](int cc, bool first) -> bool {
+    const int s = cc % kStages, b = cc & 1;
+    if (!mbar_wait(&bar->v_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
+    const uint32_t vb = v_addr + s * S::kTileBytes;
+    for (int t = 0; t < 2; ++t) {
+      if (!mbar_wait(&bar->p_ready[t][b], (uint32_t)(cc >> 1) & 1, abort_flag, state)) return false;
+      if (first && !mbar_wait(&bar->o_free[t], (i & 1) ^ 1, abort_flag, state)) return false;
+      tc_fence_after();
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off_q = (kk >> 2) * (kTileRows * 128) + (kk & 3) * 32;
-      const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-      umma_ss(tmem + S::col_s(t), sdesc_sw128(qb + off_q, 16, 1024), sdesc_sw128(kb + off_k, 16, 1024),
-              kIdescQK, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        umma_ts(tmem + S::col_o(t), tmem + S::col_s(t, b) + kk * 8,
+                sdesc_sw128(vb + kk * 2048, kBN * 128, 1024), kIdescPV, (!first || kk > 0) ? 1u : 0u);
+      umma_commit(&bar->pv_done[t][b]);
     }
-    umma_commit(&bar->s_full[t]);
+    umma_commit(&bar->v_empty[s]);
+    return true;
   };
   for (;;) {
     const int slot = i & 3;
@@ -232,24 +248,17 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
     const Item it = decode_item(p, seqs, items, idx);
     const int n_tiles = it.kt_hi - it.kt_lo + 1;
     if (!(ok = mbar_wait(&bar->q_full, i & 1, abort_flag, state))) break;
-    for (int j = 0; j < n_tiles && ok; ++j) {
-      const int s = c % kStages;
-      if (!(ok = mbar_wait(&bar->k_full[s], (uint32_t)(c / kStages) & 1, abort_flag, state))) break;
-      tc_fence_after();
-      for (int t = 0; t < 2; ++t) {
-        if (j > 0 && !(ok = issue_pv(t, c - 1, j == 1))) break;
-        issue_s(t, c);
+    if (!(ok = issue_s(c))) break;
+    if (n_tiles == 1) umma_commit(&bar->q_empty);
+    for (int j = 0; j < n_tiles; ++j) {
+      if (j + 1 < n_tiles) {
+        if (!(ok = issue_s(c + j + 1))) break;
+        if (j + 2 == n_tiles) umma_commit(&bar->q_empty);
       }
-      if (!ok) break;
-      umma_commit(&bar->k_empty[s]);
-      if (j > 0) umma_commit(&bar->v_empty[(c - 1) % kStages]);
-      if (j == n_tiles - 1) umma_commit(&bar->q_empty);
-      ++c;
+      if (!(ok = issue_pv(c + j, j == 0))) break;
     }
     if (!ok) break;
-    for (int t = 0; t < 2 && ok; ++t) ok = issue_pv(t, c - 1, n_tiles == 1);
-    if (!ok) break;
-    umma_commit(&bar->v_empty[(c - 1) % kStages]);
+    c += n_tiles;
     ++i;
   }
   // every MMA issued by this thread must finish before TMEM is released
@@ -267,7 +276,7 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
   const int q4 = warp & 3;         // TMEM lane quadrant of this warp
   const int row = q4 * 32 + lane;
   const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
-  const uint32_t t_s = t_lane + S::col_s(tq), t_o = t_lane + S::col_o(tq);
+  const uint32_t t_o = t_lane + S::col_o(tq);
   const float sl2 = p.scale_log2;
   int i = 0, c = 0;
   for (;;) {
@@ -287,7 +296,9 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      if (!(ok = warp_wait(&bar->s_full[tq], c & 1, abort_flag, state))) break;
+      const int b = c & 1;
+      const uint32_t t_s = t_lane + S::col_s(tq, b);
+      if (!(ok = warp_wait(&bar->s_full[tq][b], (uint32_t)(c >> 1) & 1, abort_flag, state))) break;
       tc_fence_after();
       float s[kBN];
 #pragma unroll
@@ -313,12 +324,14 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = mx * sl2;  // -inf stays -inf (scale > 0)
       const bool grow = m_new > m_used + kRescaleThreshold;
-      // O_t holds earlier tiles' sums scaled by m_used.  The PV that last wrote it has
-      // completed: it was issued before this tile's S, whose completion we waited for.
-      // TMEM loads/stores need the whole warp, so the warp rescales when any row must,
-      // with factor 1 for the others.
+      // O_t holds earlier tiles' sums scaled by m_used; the last PV into it (tile c - 1)
+      // must land before O_t is rescaled.  TMEM loads/stores need the whole warp, so the
+      // warp rescales when any row must, with factor 1 for the others.
       const bool rescale = grow && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, rescale)) {
+        const int pc = c - 1;  // rescale implies an earlier tile of this item: pc >= 0
+        if (!(ok = warp_wait(&bar->pv_done[tq][pc & 1], (uint32_t)(pc >> 1) & 1, abort_flag, state))) break;
+        tc_fence_after();
         const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.0f;
 #pragma unroll
         for (int cc = 0; cc < D / 16; ++cc) {
@@ -350,12 +363,12 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
       l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bar->p_ready[tq]);
+      mbar_arrive(&bar->p_ready[tq][b]);
       ++c;
     }
     if (!ok) break;
     // epilogue: the item's last PV into O_t
-    if (!warp_wait(&bar->pv_done[tq], (c - 1) & 1, abort_flag, state)) break;
+    if (!warp_wait(&bar->pv_done[tq][(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, state)) break;
     tc_fence_after();
     const float inv_l = (valid && l > 0.f) ? 1.f / l : 0.f;
     const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
@@ -421,9 +434,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar->v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&bar->s_full[t], 1);
-      mbar_init(&bar->p_ready[t], 128);
-      mbar_init(&bar->pv_done[t], 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&bar->s_full[t][b], 1);
+        mbar_init(&bar->p_ready[t][b], 128);
+        mbar_init(&bar->pv_done[t][b], 1);
+      }
       mbar_init(&bar->o_free[t], 128);
     }
     mbar_init(&bar->mma_done, 1);

@@ -9,24 +9,21 @@
 // Work item = two 128-row query tiles of one (sequence, KV head): each tile packs the G
 // query heads of the KV head over 128/G consecutive positions (GQA group packing), and the
 // two tiles cover 256/G consecutive positions.  Both tiles share every K/V tile load.
-// Key tiles hold BN = 64 keys.  Each query tile owns two S buffers in TMEM, so the tensor
-// core computes S(j+1) while the softmax warps work on S(j).
 //
 // One persistent CTA per SM, 384 threads (three warpgroups; one warp of each per SM
 // sub-partition, so the softmax warps can hold a 128-column S row in registers):
 //   warp 0      producer: takes the next item of the longest-first list (atomic counter),
 //               loads both Q tiles once, then streams K and V tiles page by page through TMA
-//               (a tile of BN = 64 keys is BN/P pages resolved through the head's page table)
-//   warp 1      MMA issuer (one thread): for key tile j, S_t(j+1) = Q_t K(j+1)^T for both
-//               query tiles, then O_t += P_t(j) V(j) as each tile's P becomes ready
+//               (a tile of BN = 128 keys is BN/P pages resolved through the head's page table)
+//   warp 1      MMA issuer (one thread): for key tile j, per query tile t,
+//               O_t += P_t(j-1) V(j-1) then S_t(j) = Q_t K(j)^T, all into TMEM
 //   warps 2, 3  idle (they hand their registers to the softmax warpgroups)
 //   warps 4..7  softmax of query tile 0, warps 8..11 softmax of query tile 1: one thread per
 //               row; fp32 online softmax in the exp2 domain, O rescaled only when the row
 //               maximum grows by more than 2^8; P (bf16) overwrites its S columns in TMEM;
 //               the epilogue normalises O and writes bf16 out, fp32 lse and visited counts.
-// P_t(j) is written as bf16 over the first half of the S buffer it came from; S_t(j+2)
-// reuses that buffer only after PV_t(j) has been issued (tcgen05 ops of one thread run in
-// issue order).
+// The two query tiles' chains (S -> softmax -> PV -> next S) interleave on the tensor core:
+// while one tile's warpgroup runs its softmax, the other tile's MMAs run.
 #include "device_common.cuh"
 
 namespace skv {
@@ -34,8 +31,8 @@ namespace skv {
 namespace {
 
 constexpr int kTileRows = 128;  // rows of one query tile (one TMEM accumulator)
-constexpr int kBN = 64;         // keys of one key tile
-constexpr int kStages = 4;      // K and V ring depth
+constexpr int kBN = 128;        // keys of one key tile
+constexpr int kStages = 2;      // K and V ring depth
 constexpr int kThreads = 384;
 // Registers per thread: 168 at launch (65536 / 384, and 3 warps x 168 x 32 fit one SM
 // sub-partition's 16384); warpgroup 0 drops to 72 and the two softmax warpgroups rise to
@@ -52,16 +49,15 @@ struct Smem {
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   static constexpr int kBytes = 1024 + kBarOff + 512;
-  // TMEM columns: S buffer b of query tile t at 128 t + 64 b, O_t at 256 + 128 t
-  static constexpr uint32_t col_s(int t, int b) { return 128u * t + 64u * b; }
+  // TMEM columns: S_t at 128 t, O_t at 256 + 128 t
+  static constexpr uint32_t col_s(int t) { return 128u * t; }
   static constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
 };
 
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2][2], p_ready[2][2], pv_done[2][2];  // [query tile][S buffer]
-  uint64_t o_free[2];
+  uint64_t s_full[2], p_ready[2], pv_done[2], o_free[2];
   uint64_t mma_done;
   uint64_t sched_full[4], sched_empty[4];
   int sched[4];
@@ -189,8 +185,6 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
 }
 
 // ---------------------------------------------------------------------------- MMA thread
-// Key tile counter c runs over every tile this CTA processes; tile c uses K/V stage
-// c % kStages and S buffer c & 1 of each query tile.
 template <int D>
 __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, const PrefillSeq *seqs, const int2 *items,
                                          uint8_t *q_s, uint8_t *k_s, uint8_t *v_s, uint32_t tmem, int32_t *state,
@@ -198,46 +192,40 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
   using S = Smem<D>;
   constexpr uint32_t kIdescQK = idesc_bf16(kTileRows, kBN, 0, 0);
   constexpr uint32_t kIdescPV = idesc_bf16(kTileRows, D, 0, 1);
-  const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
+  // Matrix descriptors differ only in their low word (start address and leading byte
+  // offset); the high word (stride 1024 B, version 1, 128-byte swizzle) is shared.
+  constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+  auto desc = [](uint32_t lo) -> uint64_t { return ((uint64_t)kHi << 32) | lo; };
+  const uint32_t q_lo = (smem_u32(q_s) >> 4) | (1u << 16);
+  const uint32_t k_lo = (smem_u32(k_s) >> 4) | (1u << 16);
+  const uint32_t v_lo = (smem_u32(v_s) >> 4) | ((uint32_t)(kBN * 128 >> 4) << 16);
   int i = 0, c = 0;
   bool ok = true;
-  // S_t(cc) = Q_t K(cc)^T for both query tiles, then release K stage
-  auto issue_s = [&](int cc) -> bool {
+  // O_t += P_t(cc) V(cc); the first PV of an item overwrites O_t
+  auto issue_pv = [&](int t, int cc, bool first, bool last) -> bool {
     const int s = cc % kStages;
-    if (!mbar_wait(&bar->k_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
+    if (!mbar_wait(&bar->p_ready[t], cc & 1, abort_flag, state)) return false;
+    if (t == 0 && !mbar_wait(&bar->v_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
+    if (first && !mbar_wait(&bar->o_free[t], (i & 1) ^ 1, abort_flag, state)) return false;
     tc_fence_after();
-    const uint32_t kb = k_addr + s * S::kTileBytes;
-    for (int t = 0; t < 2; ++t) {
-      const uint32_t qb = q_addr + t * S::kQTileBytes;
+    const uint32_t vb = v_lo + s * (S::kTileBytes >> 4);
+    const uint32_t d_o = tmem + S::col_o(t), a_p = tmem + S::col_s(t);
+    umma_ts(d_o, a_p, desc(vb), kIdescPV, first ? 0u : 1u);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off_q = (kk >> 2) * (kTileRows * 128) + (kk & 3) * 32;
-        const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-        umma_ss(tmem + S::col_s(t, cc & 1), sdesc_sw128(qb + off_q, 16, 1024), sdesc_sw128(kb + off_k, 16, 1024),
-                kIdescQK, kk > 0 ? 1u : 0u);
-      }
-      umma_commit(&bar->s_full[t][cc & 1]);
-    }
-    umma_commit(&bar->k_empty[s]);
+    for (int kk = 1; kk < kBN / 16; ++kk) umma_ts(d_o, a_p + kk * 8, desc(vb + kk * 128), kIdescPV, 1u);
+    if (last) umma_commit(&bar->pv_done[t]);
     return true;
   };
-  // O_t += P_t(cc) V(cc) for both query tiles (the first tile of an item overwrites O_t)
-  auto issue_pv = [&](int cc, bool first) -> bool {
-    const int s = cc % kStages, b = cc & 1;
-    if (!mbar_wait(&bar->v_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
-    const uint32_t vb = v_addr + s * S::kTileBytes;
-    for (int t = 0; t < 2; ++t) {
-      if (!mbar_wait(&bar->p_ready[t][b], (uint32_t)(cc >> 1) & 1, abort_flag, state)) return false;
-      if (first && !mbar_wait(&bar->o_free[t], (i & 1) ^ 1, abort_flag, state)) return false;
-      tc_fence_after();
+  // S_t(cc) = Q_t K(cc)^T
+  auto issue_s = [&](int t, int cc) {
+    const uint32_t kb = k_lo + (cc % kStages) * (S::kTileBytes >> 4);
+    const uint32_t qb = q_lo + t * (S::kQTileBytes >> 4);
+    const uint32_t d_s = tmem + S::col_s(t);
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
-        umma_ts(tmem + S::col_o(t), tmem + S::col_s(t, b) + kk * 8,
-                sdesc_sw128(vb + kk * 2048, kBN * 128, 1024), kIdescPV, (!first || kk > 0) ? 1u : 0u);
-      umma_commit(&bar->pv_done[t][b]);
-    }
-    umma_commit(&bar->v_empty[s]);
-    return true;
+    for (int kk = 0; kk < D / 16; ++kk)
+      umma_ss(d_s, desc(qb + (kk >> 2) * (kTileRows * 128 >> 4) + (kk & 3) * 2),
+              desc(kb + (kk >> 2) * (kBN * 128 >> 4) + (kk & 3) * 2), kIdescQK, kk > 0 ? 1u : 0u);
+    umma_commit(&bar->s_full[t]);
   };
   for (;;) {
     const int slot = i & 3;
@@ -248,17 +236,24 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
     const Item it = decode_item(p, seqs, items, idx);
     const int n_tiles = it.kt_hi - it.kt_lo + 1;
     if (!(ok = mbar_wait(&bar->q_full, i & 1, abort_flag, state))) break;
-    if (!(ok = issue_s(c))) break;
-    if (n_tiles == 1) umma_commit(&bar->q_empty);
-    for (int j = 0; j < n_tiles; ++j) {
-      if (j + 1 < n_tiles) {
-        if (!(ok = issue_s(c + j + 1))) break;
-        if (j + 2 == n_tiles) umma_commit(&bar->q_empty);
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      const int s = c % kStages;
+      if (!(ok = mbar_wait(&bar->k_full[s], (uint32_t)(c / kStages) & 1, abort_flag, state))) break;
+      tc_fence_after();
+      for (int t = 0; t < 2; ++t) {
+        if (j > 0 && !(ok = issue_pv(t, c - 1, j == 1, false))) break;
+        issue_s(t, c);
       }
-      if (!(ok = issue_pv(c + j, j == 0))) break;
+      if (!ok) break;
+      umma_commit(&bar->k_empty[s]);
+      if (j > 0) umma_commit(&bar->v_empty[(c - 1) % kStages]);
+      if (j == n_tiles - 1) umma_commit(&bar->q_empty);
+      ++c;
     }
     if (!ok) break;
-    c += n_tiles;
+    for (int t = 0; t < 2 && ok; ++t) ok = issue_pv(t, c - 1, n_tiles == 1, true);
+    if (!ok) break;
+    umma_commit(&bar->v_empty[(c - 1) % kStages]);
     ++i;
   }
   // every MMA issued by this thread must finish before TMEM is released
@@ -276,7 +271,7 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
   const int q4 = warp & 3;         // TMEM lane quadrant of this warp
   const int row = q4 * 32 + lane;
   const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
-  const uint32_t t_o = t_lane + S::col_o(tq);
+  const uint32_t t_s = t_lane + S::col_s(tq), t_o = t_lane + S::col_o(tq);
   const float sl2 = p.scale_log2;
   int i = 0, c = 0;
   for (;;) {
@@ -296,14 +291,12 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const int b = c & 1;
-      const uint32_t t_s = t_lane + S::col_s(tq, b);
-      if (!(ok = warp_wait(&bar->s_full[tq][b], (uint32_t)(c >> 1) & 1, abort_flag, state))) break;
+      if (!(ok = warp_wait(&bar->s_full[tq], c & 1, abort_flag, state))) break;
       tc_fence_after();
+      static_assert(kBN == 128, "128-key tiles");
       float s[kBN];
 #pragma unroll
-      for (int cc = 0; cc < kBN / 16; ++cc)
-        tmem_ld16(t_s + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[cc * 16]));
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(t_s + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
       tmem_ld_wait();
       const int k0 = (it.kt_lo + j) * kBN;
       if (k0 < lo || k0 + kBN - 1 > pq) {
@@ -315,60 +308,57 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
       }
       float mx8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+      for (int e = 0; e < 8; ++e) mx8[e] = fmax3(s[e], s[8 + e], s[16 + e]);
 #pragma unroll
-      for (int jj = 8; jj < kBN; jj += 8)
+      for (int r = 0; r < 7; ++r)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], s[jj + e]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_new = mx * sl2;  // -inf stays -inf (scale > 0)
+        for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], s[24 + 16 * r + e], s[32 + 16 * r + e]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], s[120 + e]);
+      const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+      const float m_new = mx * sl2;
       const bool grow = m_new > m_used + kRescaleThreshold;
-      // O_t holds earlier tiles' sums scaled by m_used; the last PV into it (tile c - 1)
-      // must land before O_t is rescaled.  TMEM loads/stores need the whole warp, so the
-      // warp rescales when any row must, with factor 1 for the others.
       const bool rescale = grow && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, rescale)) {
-        const int pc = c - 1;  // rescale implies an earlier tile of this item: pc >= 0
-        if (!(ok = warp_wait(&bar->pv_done[tq][pc & 1], (uint32_t)(pc >> 1) & 1, abort_flag, state))) break;
-        tc_fence_after();
         const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.0f;
 #pragma unroll
-        for (int cc = 0; cc < D / 16; ++cc) {
-          uint32_t o[16];
-          tmem_ld16(t_o + cc * 16, o);
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(t_o + cc * 32, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st16(t_o + cc * 16, o);
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(t_o + cc * 32, o);
         }
         l *= alpha;
       }
       if (grow) m_used = m_new;
-      // P = exp2(s * scale_log2 - m_used), written as bf16 pairs over the S columns
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int cc = 0; cc < kBN / 32; ++cc) {
-        uint32_t pk[16];
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = fast_exp2(fmaf(s[cc * 32 + 2 * e], sl2, neg_m));
-          const float b2 = fast_exp2(fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m));
-          rs[e & 3] += a + b2;
-          pk[e] = pack_bf16x2(a, b2);
+        for (int e = 0; e < 32; ++e) {
+          const float2 x = ffma2(make_float2(s[cc * 64 + 2 * e], s[cc * 64 + 2 * e + 1]), c2, nm2);
+          const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          acc[e & 3] = fadd2(acc[e & 3], pe);
+          pk[e] = pack_bf16x2(pe.x, pe.y);
         }
-        tmem_st16(t_s + cc * 16, pk);
+        tmem_st32(t_s + cc * 32, pk);
       }
-      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+      const float2 a = fadd2(a01, a23);
+      l += a.x + a.y;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bar->p_ready[tq][b]);
+      mbar_arrive(&bar->p_ready[tq]);
       ++c;
     }
     if (!ok) break;
     // epilogue: the item's last PV into O_t
-    if (!warp_wait(&bar->pv_done[tq][(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, state)) break;
+    if (!warp_wait(&bar->pv_done[tq], (uint32_t)i & 1, abort_flag, state)) break;  // one phase per item
     tc_fence_after();
     const float inv_l = (valid && l > 0.f) ? 1.f / l : 0.f;
     const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
@@ -434,11 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar->v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&bar->s_full[t][b], 1);
-        mbar_init(&bar->p_ready[t][b], 128);
-        mbar_init(&bar->pv_done[t][b], 1);
-      }
+      mbar_init(&bar->s_full[t], 1);
+      mbar_init(&bar->p_ready[t], 128);
+      mbar_init(&bar->pv_done[t], 1);
       mbar_init(&bar->o_free[t], 128);
     }
     mbar_init(&bar->mma_done, 1);

@@ -24,7 +24,7 @@ namespace {
 
 constexpr int kPrefillTileRows = 128;  // rows of one prefill query tile (G heads x 128/G positions)
 constexpr int kPrefillItemRows = 256;  // rows of one prefill work item (two query tiles)
-constexpr int kPrefillKeyTile = 64;    // keys of a prefill key tile
+constexpr int kPrefillKeyTile = 128;   // keys of a prefill key tile
 constexpr int kDecodeStageKeys = 64;   // keys of a decode pipeline stage
 constexpr int kMaxSplits = 32;         // most splits one decode head is cut into
 constexpr int kMaxPairs = 8192;        // (sequence, KV head) pairs of one append

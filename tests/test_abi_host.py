@@ -114,7 +114,7 @@ def test_plan_matches_oracle_lpt_order(name):
     for layer in range(w.layers):
         got, tile_pos, key_tile = h.plan_prefill(layer, qs, ql)
         want = orc.lpt_items(qs, ql, w.classes[layer], w.window, tile_pos, key_tile)
-        assert tile_pos == 256 // w.group and key_tile == 64
+        assert tile_pos == 256 // w.group and key_tile == 128
         assert np.array_equal(got, want)
 
 

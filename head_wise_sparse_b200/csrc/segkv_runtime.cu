@@ -558,3 +558,152 @@ int segkv_device_status(segkv_t *h, void *stream) {
 }
 
 }  // extern "C"
+
+// ============================================================================== decode without allocation
+// For callers that cannot hand the library a workspace: the split partials, the scheduler
+// counter and the per-call metadata live in a fixed scratch array that this file owns.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 64u << 20;  // device scratch, held by every GPU that loads the library
+constexpr size_t kNoAllocMetaBytes = 1u << 20;      // host-side metadata, pageable
+constexpr int kNoAllocMaxDevices = 64;
+constexpr int kNoAllocMaxSeqSlots = 1 << 16;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+unsigned char g_noalloc_meta[kNoAllocMetaBytes];
+uint64_t g_noalloc_seen[kNoAllocMaxSeqSlots / 64];
+void *g_noalloc_dev_ptr[kNoAllocMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once per device.
+int noalloc_scratch(segkv_t *h, void **ptr) {
+  int dev = 0;
+  SEGKV_CUDA(h, "cudaGetDevice", cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) {
+    h->last_error = "fixed scratch: device index beyond the supported 64";
+    return SEGKV_ERR_UNSUPPORTED;
+  }
+  if (!g_noalloc_dev_ptr[dev]) {
+    void *p = nullptr;
+    SEGKV_CUDA(h, "scratch symbol address", cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_dev_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_dev_ptr[dev];
+  return SEGKV_OK;
+}
+
+}  // namespace
+
+extern "C" int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
+                                         const int32_t *q_pos, const void *q, float softmax_scale, int num_splits,
+                                         void *out, float *lse, uint64_t *visited, void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= h->cfg.num_layers || nseq < 1 || nseq > h->cfg.max_seqs || !seq_ids || !q_pos ||
+      num_splits < 0)
+    return SEGKV_ERR_INVALID_ARG;
+  if (h->cfg.max_seqs > kNoAllocMaxSeqSlots) return SEGKV_ERR_UNSUPPORTED;
+  if (h->G > 16) return SEGKV_ERR_UNSUPPORTED;
+  if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4)) return SEGKV_ERR_INVALID_ARG;
+  // distinct sequence ids (a fixed bitmap, cleared again before returning)
+  int rc = SEGKV_OK;
+  int b_seen = 0;
+  for (; b_seen < nseq; ++b_seen) {
+    const int s = seq_ids[b_seen];
+    if (s < 0 || s >= h->cfg.max_seqs || (g_noalloc_seen[s >> 6] >> (s & 63) & 1)) {
+      rc = SEGKV_ERR_INVALID_ARG;
+      break;
+    }
+    g_noalloc_seen[s >> 6] |= 1ull << (s & 63);
+  }
+  for (int b = 0; b < b_seen; ++b) g_noalloc_seen[seq_ids[b] >> 6] &= ~(1ull << (seq_ids[b] & 63));
+  if (rc) return rc;
+  const int P = h->cfg.page_size, H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
+  const bool has_local = layer_has_local(h, layer);
+  long long total_pages = 0;
+  int max_pages = 0;
+  for (int b = 0; b < nseq; ++b) {
+    const int len = h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]];
+    if (q_pos[b] < 0 || q_pos[b] >= len) return SEGKV_ERR_INVALID_ARG;
+    if (has_local && !ring_covers(h, len, q_pos[b])) return SEGKV_ERR_RING_TOO_SMALL;
+    for (int k = 0; k < H; ++k) {
+      const int lo = h->cls[layer * H + k] ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
+      const int n = q_pos[b] / P - lo / P + 1;
+      total_pages += n;
+      max_pages = std::max(max_pages, n);
+    }
+  }
+  if ((rc = ensure_device_state(h))) return rc;
+  // the same split rule as segkv_decode_attn
+  const int pps = kDecodeStageKeys / P;
+  int split;
+  if (num_splits > 0) {
+    split = ceil_div(max_pages, std::min(num_splits, kMaxSplits));
+  } else {
+    const long long target = std::max<long long>(1, total_pages / (8LL * h->num_sms));
+    split = 1;
+    while (2LL * split <= target && split < 256) split *= 2;
+  }
+  split = std::max(split, ceil_div(max_pages, kMaxSplits));
+  split = ceil_div(split, pps) * pps;
+  const int max_splits = ceil_div(max_pages, split);
+  long long n_items = 0;
+  for (int b = 0; b < nseq; ++b)
+    for (int k = 0; k < H; ++k) {
+      const int lo = h->cls[layer * H + k] ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
+      n_items += ceil_div(q_pos[b] / P - lo / P + 1, split);
+    }
+  const size_t nsplit_off = kHeaderBytes + sizeof(DecodeSeq) * nseq;
+  const size_t items_off = align_up(nsplit_off + 4 * (size_t)nseq * H, 16);
+  const size_t meta_bytes = items_off + 8 * (size_t)n_items;
+  const size_t part_o_off = align_up(meta_bytes, 256);
+  const size_t part_lse_off = part_o_off + align_up(4 * (size_t)nseq * Hq * max_splits * D, 256);
+  const size_t need = part_lse_off + 4 * (size_t)nseq * Hq * max_splits;
+  if (meta_bytes > kNoAllocMetaBytes || need > kNoAllocScratchBytes) {
+    h->last_error = "decode needs " + std::to_string(need) + " bytes of scratch (metadata " +
+                    std::to_string(meta_bytes) + "); the fixed scratch holds " +
+                    std::to_string(kNoAllocScratchBytes) + " (metadata " + std::to_string(kNoAllocMetaBytes) + ")";
+    return SEGKV_ERR_WORKSPACE;
+  }
+  void *scratch = nullptr;
+  if ((rc = noalloc_scratch(h, &scratch))) return rc;
+  // metadata: zeroed header (the scheduler counter), sequence table, split counts, items
+  unsigned char *host = g_noalloc_meta;
+  std::memset(host, 0, items_off);
+  DecodeSeq *ds = reinterpret_cast<DecodeSeq *>(host + kHeaderBytes);
+  int32_t *ns = reinterpret_cast<int32_t *>(host + nsplit_off);
+  int2 *it = reinterpret_cast<int2 *>(host + items_off);
+  long long w = 0;
+  for (int b = 0; b < nseq; ++b) {
+    ds[b] = DecodeSeq{seq_ids[b], q_pos[b], h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]], 0};
+    for (int k = 0; k < H; ++k) {
+      const bool global = h->cls[layer * H + k] != 0;
+      const int lo = global ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
+      const int n = ceil_div(q_pos[b] / P - lo / P + 1, split);
+      ns[(size_t)b * H + k] = n;
+      for (int s = 0; s < n; ++s) it[w++] = make_int2(b, (int)make_item_w1(global, k, s));
+    }
+  }
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // a copy from pageable memory has read the host buffer when it returns
+  SEGKV_CUDA(h, "scratch metadata upload", cudaMemcpyAsync(scratch, host, meta_bytes, cudaMemcpyHostToDevice, st));
+  DecodeLaunch p;
+  p.g = geom(h);
+  p.layer = layer;
+  p.nseq = nseq;
+  p.n_items = (int)n_items;
+  p.split_pages = split;
+  p.max_splits = max_splits;
+  p.grid = std::min<int>((int)n_items, h->num_sms);
+  p.ws_meta = scratch;
+  p.nsplit_off = (int)nsplit_off;
+  p.items_off = (int)items_off;
+  p.part_o = reinterpret_cast<float *>(static_cast<char *>(scratch) + part_o_off);
+  p.part_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) + part_lse_off);
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.visited = reinterpret_cast<unsigned long long *>(visited);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  SEGKV_CUDA(h, "decode launch", launch_decode(p, h->kmap, h->vmap, st));
+  return SEGKV_OK;
+}

@@ -25,6 +25,7 @@ EXPORTS = [
     "segkv_create", "segkv_destroy", "segkv_ring_pages", "segkv_max_lp", "segkv_seq_len", "segkv_pages_used",
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
     "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
+    "segkv_decode_attn_noalloc",
 ]
 
 
@@ -71,6 +72,7 @@ def lib():
         L.segkv_plan_prefill.argtypes = [P, I, I, P, P, P, I64, ctypes.POINTER(I64), ctypes.POINTER(I),
                                          ctypes.POINTER(I)]
         L.segkv_decode_attn.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P, SZ, P]
+        L.segkv_decode_attn_noalloc.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P]
         L.segkv_device_status.argtypes = [P, P]
         L.segkv_last_error.argtypes = [P]
         L.segkv_last_error.restype = ctypes.c_char_p
@@ -172,6 +174,13 @@ class Handle:
         s, qp = _i32(seq_ids), _i32(q_pos)
         return lib().segkv_decode_attn(self.h, layer, len(s), _p(s), _p(qp), _dptr(q), float(scale), int(num_splits),
                                        _dptr(out), _dptr(lse), _dptr(visited), _dptr(ws), ws_bytes, _stream(stream))
+
+    def decode_noalloc(self, layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, stream=None) -> int:
+        """segkv_decode_attn_noalloc: decode without a workspace, on the library's fixed scratch."""
+        s, qp = _i32(seq_ids), _i32(q_pos)
+        return lib().segkv_decode_attn_noalloc(self.h, layer, len(s), _p(s), _p(qp), _dptr(q), float(scale),
+                                               int(num_splits), _dptr(out), _dptr(lse), _dptr(visited),
+                                               _stream(stream))
 
     def plan_prefill(self, layer, q_start, q_len):
         """Longest-processing-time-first list as int32 rows (seq index, KV head, tile, cost)."""

@@ -160,6 +160,28 @@ int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
                       const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
                       void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * Decode with no caller workspace and no allocation.  The pages have no counterpart to
+ * this entry point; it exists for callers that cannot give the library device memory:
+ * a serving engine that reserved the whole device for its own allocator at start-up, or
+ * code running under a fixed memory budget where a cudaMalloc would fail or is not
+ * allowed.  Arguments, results and errors are those of segkv_decode_attn, minus ws.
+ *   Scratch: the split partials, the work list and the scheduler counter live in one
+ *   fixed array of 64 MiB inside libsegkv.so (every GPU that loads the library holds it
+ *   until the process exits); per-call metadata is staged in a fixed 1 MiB host buffer.
+ *   A call that would need more returns SEGKV_ERR_WORKSPACE and names the sizes in
+ *   segkv_last_error.  Nothing is allocated: no cudaMalloc, cudaFree or cudaHostAlloc.
+ *   The first call on a device looks up the array's device address (once per device);
+ *   make that first call before any stream capture.
+ *   Every call shares the one array and the scheduler counter is re-zeroed by each call's
+ *   metadata copy, so calls that overlap on the GPU (different streams, or different
+ *   handles) race and give wrong results: issue them one after another on one stream.
+ *   Not thread-safe.
+ */
+int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,
+                              const void *q, float softmax_scale, int num_splits, void *out, float *lse,
+                              uint64_t *visited, void *stream);
+
 /* Synchronizes `stream`, reads the device error word, clears it and returns it
  * (SEGKV_OK, SEGKV_ERR_DEVICE_BOUNDS or SEGKV_ERR_DEVICE_TIMEOUT), or SEGKV_ERR_CUDA. */
 int segkv_device_status(segkv_t *h, void *stream);

@@ -13,7 +13,9 @@
 // One persistent CTA per SM, 384 threads (three warpgroups; one warp of each per SM
 // sub-partition, so the softmax warps can hold a 128-column S row in registers):
 //   warp 0      producer: takes the next item of the longest-first list (atomic counter),
-//               loads both Q tiles once, then streams K and V tiles page by page through TMA
+//               decodes it once into a shared-memory ring the other roles read, pulls the
+//               following item's Q rows into L2, loads both Q tiles, then streams K and V
+//               tiles page by page through TMA
 //               (a tile of BN = 128 keys is BN/P pages resolved through the head's page table)
 //   warp 1      MMA issuer (one thread): for key tile j, per query tile t,
 //               O_t += P_t(j-1) V(j-1) then S_t(j) = Q_t K(j)^T, all into TMEM
@@ -48,10 +50,15 @@ struct Smem {
   static constexpr int kKOff = 2 * kQTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  static constexpr int kBytes = 1024 + kBarOff + 512;
+  static constexpr int kBytes = 1024 + kBarOff + 1024;
   // TMEM columns: S_t at 128 t, O_t at 256 + 128 t
   static constexpr uint32_t col_s(int t) { return 128u * t; }
   static constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
+};
+
+struct Item {
+  int b, h, t, q_first, q_last, lo_min, kt_lo, kt_hi, seq_id, kv_len, q_row;
+  bool global;
 };
 
 struct Bars {
@@ -61,14 +68,11 @@ struct Bars {
   uint64_t mma_done;
   uint64_t sched_full[4], sched_empty[4];
   int sched[4];
+  Item sched_item[4];  // the producer decodes each item once; consumers read it here
   uint32_t tmem_base;
   int abort_flag;
 };
 
-struct Item {
-  int b, h, t, q_first, q_last, lo_min, kt_lo, kt_hi, seq_id, kv_len, q_row;
-  bool global;
-};
 
 // Item = (sequence b, KV head h, tile pair t): positions [q_start + 2 t tp, ...) of the
 // sequence's queries, tp = 128 / G positions per query tile.
@@ -110,19 +114,31 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
   const int P = p.g.page, PPT = kBN / P;
   int i = 0, c = 0;
   bool ok = true, q_loaded = false;
+  // next item index, fetched one item ahead so its Q rows can be pulled into L2 early
+  auto fetch = [&]() -> int {
+    int v = 0;
+    if (lane == 0) v = atomicAdd(sched_next, 1);
+    v = __shfl_sync(0xffffffffu, v, 0);
+    return v < p.n_items ? v : -1;
+  };
+  int idx = fetch();
   for (;;) {
-    int idx = 0;
-    if (lane == 0) idx = atomicAdd(sched_next, 1);
-    idx = __shfl_sync(0xffffffffu, idx, 0);
-    if (idx >= p.n_items) idx = -1;
     const int slot = i & 3;
+    Item it;
+    if (idx >= 0) it = decode_item(p, seqs, items, idx);
     if (!(ok = warp_wait(&bar->sched_empty[slot], ((i >> 2) & 1) ^ 1, abort_flag, state))) break;
     if (lane == 0) {
       bar->sched[slot] = idx;
+      if (idx >= 0) bar->sched_item[slot] = it;
       mbar_arrive(&bar->sched_full[slot]);
     }
     if (idx < 0) break;
-    const Item it = decode_item(p, seqs, items, idx);
+    const int next = fetch();
+    if (next >= 0 && lane == 0) {
+      const Item nt = decode_item(p, seqs, items, next);
+      for (int t = 0; t < 2; ++t)
+        for (int hh = 0; hh < S::kHalves; ++hh) tma_prefetch_l2_3d(&qmap, hh * 64, nt.h * G, nt.q_row + t * p.tile_pos);
+    }
     if (!(ok = warp_wait(&bar->q_empty, (i & 1) ^ 1, abort_flag, state))) break;
     if (lane == 0) {
       mbar_expect_tx(&bar->q_full, 2 * S::kQTileBytes);
@@ -173,6 +189,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
     }
     if (!ok) break;
     ++i;
+    idx = next;
   }
   // drain: no copy of this CTA may still be in flight when it exits
   for (int k = c - 1; k >= 0 && k >= c - kStages; --k) {
@@ -231,9 +248,9 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
     const int slot = i & 3;
     if (!(ok = mbar_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state))) break;
     const int idx = bar->sched[slot];
+    const Item it = bar->sched_item[slot];
     mbar_arrive(&bar->sched_empty[slot]);
     if (idx < 0) break;
-    const Item it = decode_item(p, seqs, items, idx);
     const int n_tiles = it.kt_hi - it.kt_lo + 1;
     if (!(ok = mbar_wait(&bar->q_full, i & 1, abort_flag, state))) break;
     for (int j = 0; j < n_tiles && ok; ++j) {
@@ -278,10 +295,10 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
     const int slot = i & 3;
     if (!warp_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state)) break;
     const int idx = bar->sched[slot];
+    const Item it = bar->sched_item[slot];
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar->sched_empty[slot]);
     if (idx < 0) break;
-    const Item it = decode_item(p, seqs, items, idx);
     const int n_tiles = it.kt_hi - it.kt_lo + 1;
     const int pos_local = tq * p.tile_pos + row / G, g = row % G;
     const int p_raw = it.q_first + pos_local;
@@ -300,11 +317,12 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
       tmem_ld_wait();
       const int k0 = (it.kt_lo + j) * kBN;
       if (k0 < lo || k0 + kBN - 1 > pq) {
+        // keep columns a..b of this tile: one unsigned compare per element
+        const int a = lo - k0;
+        const unsigned span = (unsigned)(pq - lo);
 #pragma unroll
-        for (int jj = 0; jj < kBN; ++jj) {
-          const int kp = k0 + jj;
-          if (kp < lo || kp > pq) s[jj] = -INFINITY;
-        }
+        for (int jj = 0; jj < kBN; ++jj)
+          if ((unsigned)(jj - a) > span) s[jj] = -INFINITY;
       }
       float mx8[8];
 #pragma unroll
@@ -364,17 +382,17 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
     const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
     uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
 #pragma unroll
-    for (int cc = 0; cc < D / 16; ++cc) {
-      uint32_t o[16];
-      tmem_ld16(t_o + cc * 16, o);
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      tmem_ld32(t_o + cc * 32, o);
       tmem_ld_wait();
-      uint32_t w[8];
+      uint32_t w[16];
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
+      for (int e = 0; e < 16; ++e)
         w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
       if (valid) {
-        dst[cc * 2 + 0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[cc * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) dst[cc * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
       }
     }
     tc_fence_before();

@@ -63,7 +63,7 @@ struct PrefillLaunch {
   float scale_log2;
 };
 cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
-                           const CUtensorMap &vmap, cudaStream_t st);
+                           const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t st);
 int prefill_smem_bytes(int head_dim);
 
 struct DecodeLaunch {

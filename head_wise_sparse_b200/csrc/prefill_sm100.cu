@@ -18,12 +18,19 @@
 //               tiles page by page through TMA
 //               (a tile of BN = 128 keys is BN/P pages resolved through the head's page table)
 //   warp 1      MMA issuer (one thread): for key tile j, per query tile t,
-//               O_t += P_t(j-1) V(j-1) then S_t(j) = Q_t K(j)^T, all into TMEM
+//               O_t += P_t(j-1) V(j-1) in two halves of 64 keys (each issued as soon as
+//               the softmax has written that half of P_t(j-1)), then S_t(j) = Q_t K(j)^T,
+//               all into TMEM
 //   warps 2, 3  idle (they hand their registers to the softmax warpgroups)
 //   warps 4..7  softmax of query tile 0, warps 8..11 softmax of query tile 1: one thread per
 //               row; fp32 online softmax in the exp2 domain, O rescaled only when the row
-//               maximum grows by more than 2^8; P (bf16) overwrites its S columns in TMEM;
-//               the epilogue normalises O and writes bf16 out, fp32 lse and visited counts.
+//               maximum grows by more than 2^8; P (bf16) overwrites its S columns in TMEM,
+//               each half of 64 keys signalled as soon as it is stored;
+//               the epilogue reads O_t out of TMEM (and frees it for the next item at once),
+//               normalises it and writes bf16 out through a 128-byte-swizzled shared-memory
+//               buffer and TMA tile stores (64 columns at a time; scattered per-thread row
+//               stores would flood the SM's L2 request path that the K/V loads share),
+//               plus fp32 lse and visited counts.
 // The two query tiles' chains (S -> softmax -> PV -> next S) interleave on the tensor core:
 // while one tile's warpgroup runs its softmax, the other tile's MMAs run.
 #include "device_common.cuh"
@@ -36,11 +43,20 @@ constexpr int kTileRows = 128;  // rows of one query tile (one TMEM accumulator)
 constexpr int kBN = 128;        // keys of one key tile
 constexpr int kStages = 2;      // K and V ring depth
 constexpr int kThreads = 384;
-// Registers per thread: 168 at launch (65536 / 384, and 3 warps x 168 x 32 fit one SM
-// sub-partition's 16384); warpgroup 0 drops to 72 and the two softmax warpgroups rise to
-// 216, which adds up to the launch total: 128 x 72 + 256 x 216 = 384 x 168.
-constexpr int kRegsLow = 72, kRegsHigh = 216;
+// Registers per thread: 168 at launch (65536 / 384 rounded down to a multiple of 8);
+// warpgroup 0 drops to 72 and the two softmax warpgroups rise to 216, which adds up to the
+// launch total: 128 x 72 + 256 x 216 = 384 x 168 (setmaxnreg.inc can only take registers
+// the block was launched with).
+constexpr int kRegsLaunch = (65536 / kThreads) / 8 * 8;
+constexpr int kRegsLow = 72, kRegsHigh = (kRegsLaunch * kThreads - 128 * kRegsLow) / 256 / 8 * 8;
+static_assert(kRegsHigh == 216 && 128 * kRegsLow + 256 * kRegsHigh <= kRegsLaunch * kThreads,
+              "register split exceeds the launch total");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
+// One exponential pair in kEmuEvery may go to the FMA pipe (exp2_fma2) instead of the
+// MUFU; 0 keeps all of them on the MUFU.  Measured on the Mistral-shaped and 128K-chunk
+// workloads, every ratio from 1/8 to 1/2 was slower: the softmax here is bound by its
+// instruction stream and latency, not by MUFU throughput.
+constexpr int kEmuEvery = 0;
 
 template <int D>
 struct Smem {
@@ -49,7 +65,10 @@ struct Smem {
   static constexpr int kHalves = D / 64;
   static constexpr int kKOff = 2 * kQTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // output staging: one buffer of 128 rows x 64 columns (16 KiB) per softmax warpgroup
+  static constexpr int kOStageBytes = kTileRows * 128;
+  static constexpr int kOOff = kVOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kOOff + 2 * kOStageBytes;
   static constexpr int kBytes = 1024 + kBarOff + 1024;
   // TMEM columns: S_t at 128 t, O_t at 256 + 128 t
   static constexpr uint32_t col_s(int t) { return 128u * t; }
@@ -64,7 +83,7 @@ struct Item {
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_ready[2], pv_done[2], o_free[2];
+  uint64_t s_full[2], p_lo[2], p_hi[2], pv_done[2], o_free[2];
   uint64_t mma_done;
   uint64_t sched_full[4], sched_empty[4];
   int sched[4];
@@ -221,7 +240,7 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
   // O_t += P_t(cc) V(cc); the first PV of an item overwrites O_t
   auto issue_pv = [&](int t, int cc, bool first, bool last) -> bool {
     const int s = cc % kStages;
-    if (!mbar_wait(&bar->p_ready[t], cc & 1, abort_flag, state)) return false;
+    if (!mbar_wait(&bar->p_lo[t], cc & 1, abort_flag, state)) return false;
     if (t == 0 && !mbar_wait(&bar->v_full[s], (uint32_t)(cc / kStages) & 1, abort_flag, state)) return false;
     if (first && !mbar_wait(&bar->o_free[t], (i & 1) ^ 1, abort_flag, state)) return false;
     tc_fence_after();
@@ -229,7 +248,11 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
     const uint32_t d_o = tmem + S::col_o(t), a_p = tmem + S::col_s(t);
     umma_ts(d_o, a_p, desc(vb), kIdescPV, first ? 0u : 1u);
 #pragma unroll
-    for (int kk = 1; kk < kBN / 16; ++kk) umma_ts(d_o, a_p + kk * 8, desc(vb + kk * 128), kIdescPV, 1u);
+    for (int kk = 1; kk < kBN / 32; ++kk) umma_ts(d_o, a_p + kk * 8, desc(vb + kk * 128), kIdescPV, 1u);
+    if (!mbar_wait(&bar->p_hi[t], cc & 1, abort_flag, state)) return false;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = kBN / 32; kk < kBN / 16; ++kk) umma_ts(d_o, a_p + kk * 8, desc(vb + kk * 128), kIdescPV, 1u);
     if (last) umma_commit(&bar->pv_done[t]);
     return true;
   };
@@ -280,9 +303,10 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
 
 // ---------------------------------------------------------------------------- softmax warpgroups
 template <int D>
-__device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, const PrefillSeq *seqs,
-                                             const int2 *items, uint32_t tmem, int warp, int lane, int G,
-                                             int32_t *state, volatile int *abort_flag) {
+__device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const PrefillLaunch &p, Bars *bar,
+                                             const PrefillSeq *seqs, const int2 *items, uint8_t *o_stage,
+                                             uint32_t tmem, int warp, int lane, int G, int32_t *state,
+                                             volatile int *abort_flag) {
   using S = Smem<D>;
   const int tq = (warp - 4) >> 2;  // query tile of this warpgroup
   const int q4 = warp & 3;         // TMEM lane quadrant of this warp
@@ -316,7 +340,8 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
       for (int cc = 0; cc < 4; ++cc) tmem_ld32(t_s + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
       tmem_ld_wait();
       const int k0 = (it.kt_lo + j) * kBN;
-      if (k0 < lo || k0 + kBN - 1 > pq) {
+      // warp-uniform branch: only tiles that cut some row's window edge or diagonal mask
+      if (__any_sync(0xffffffffu, k0 < lo || k0 + kBN - 1 > pq)) {
         // keep columns a..b of this tile: one unsigned compare per element
         const int a = lo - k0;
         const unsigned span = (unsigned)(pq - lo);
@@ -354,49 +379,79 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // P in two halves of 64 keys; the MMA thread starts each half's PV as it lands
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const float2 x = ffma2(make_float2(s[cc * 64 + 2 * e], s[cc * 64 + 2 * e + 1]), c2, nm2);
-          const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          float2 pe;
+          if (kEmuEvery > 0 && e % (kEmuEvery > 0 ? kEmuEvery : 1) == kEmuEvery - 1)
+            pe = exp2_fma2(x);
+          else
+            pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
           acc[e & 3] = fadd2(acc[e & 3], pe);
           pk[e] = pack_bf16x2(pe.x, pe.y);
         }
         tmem_st32(t_s + cc * 32, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(cc == 0 ? &bar->p_lo[tq] : &bar->p_hi[tq]);
       }
       const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
       const float2 a = fadd2(a01, a23);
       l += a.x + a.y;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bar->p_ready[tq]);
       ++c;
     }
     if (!ok) break;
     // epilogue: the item's last PV into O_t
     if (!warp_wait(&bar->pv_done[tq], (uint32_t)i & 1, abort_flag, state)) break;  // one phase per item
     tc_fence_after();
+    uint32_t o[D];
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(t_o + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[cc * 32]));
+    tmem_ld_wait();
+    tc_fence_before();
+    mbar_arrive(&bar->o_free[tq]);  // O_t is in registers: the next item's first PV may overwrite it
     const float inv_l = (valid && l > 0.f) ? 1.f / l : 0.f;
     const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
-    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
+    // a tile whose rows are all real queries goes out through TMA; the last tile of a
+    // sequence may run past it (those rows belong to the next sequence) and is stored row
+    // by row
+    if (it.q_first + (tq + 1) * p.tile_pos - 1 <= it.q_last) {
+      uint8_t *stg = o_stage + tq * Smem<D>::kOStageBytes;
+      const bool leader = (threadIdx.x & 127) == 0;
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t o[32];
-      tmem_ld32(t_o + cc * 32, o);
-      tmem_ld_wait();
-      uint32_t w[16];
+      for (int hh = 0; hh < D / 64; ++hh) {
+        uint32_t w[32];
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-      if (valid) {
+        for (int e = 0; e < 32; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o[hh * 64 + 2 * e]) * inv_l, __uint_as_float(o[hh * 64 + 2 * e + 1]) * inv_l);
+        if (leader) bulk_wait_read_all();  // the previous store has read the buffer
+        named_bar_sync(1 + tq, 128);
+        // row r of the box at r * 128 bytes, 16-byte chunk c at (c ^ (r mod 8)): the
+        // 128-byte swizzle the output tensor map expects
 #pragma unroll
-        for (int v = 0; v < 4; ++v) dst[cc * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4 *>(stg + row * 128 + ((c ^ (row & 7)) << 4)) =
+              make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        fence_async_smem();
+        named_bar_sync(1 + tq, 128);
+        if (leader) {
+          tma_store_3d(&omap, stg, hh * 64, it.h * G, it.q_row + tq * p.tile_pos);
+          bulk_commit();
+        }
       }
+    } else if (valid) {
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
+#pragma unroll
+      for (int v = 0; v < D / 8; ++v)
+        dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l),
+                            pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l),
+                            pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l),
+                            pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
     }
-    tc_fence_before();
-    mbar_arrive(&bar->o_free[tq]);
     if (valid) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;
     if (p.visited) {
       unsigned long long cnt = valid ? (unsigned long long)(pq - lo + 1) : 0ull;
@@ -409,18 +464,21 @@ __device__ __forceinline__ void softmax_role(const PrefillLaunch &p, Bars *bar, 
     }
     ++i;
   }
+  if ((threadIdx.x & 127) == 0) bulk_wait_all();  // no store of this warpgroup outlives the CTA
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, const PrefillLaunch p) {
+                   const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
+                   const PrefillLaunch p) {
   using S = Smem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_s = base;
   uint8_t *k_s = base + S::kKOff;
   uint8_t *v_s = base + S::kVOff;
+  uint8_t *o_stage = base + S::kOOff;
   Bars *bar = reinterpret_cast<Bars *>(base + S::kBarOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -443,7 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar->s_full[t], 1);
-      mbar_init(&bar->p_ready[t], 128);
+      mbar_init(&bar->p_lo[t], 128);
+      mbar_init(&bar->p_hi[t], 128);
       mbar_init(&bar->pv_done[t], 1);
       mbar_init(&bar->o_free[t], 128);
     }
@@ -463,7 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= 4) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-    softmax_role<D>(p, bar, seqs, items, tmem, warp, lane, G, state, abort_flag);
+    if (lane == 0 && (warp & 3) == 0) tma_prefetch_desc(&omap);
+    softmax_role<D>(omap, p, bar, seqs, items, o_stage, tmem, warp, lane, G, state, abort_flag);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
@@ -486,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 int prefill_smem_bytes(int head_dim) { return head_dim == 64 ? Smem<64>::kBytes : Smem<128>::kBytes; }
 
 cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
-                           const CUtensorMap &vmap, cudaStream_t st) {
+                           const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t st) {
   static bool attr_set[2] = {false, false};
   const int smem = prefill_smem_bytes(p.g.head_dim);
   cudaError_t e;
@@ -496,14 +556,14 @@ cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, cons
         return e;
       attr_set[0] = true;
     }
-    prefill_kernel<64><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, p);
+    prefill_kernel<64><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, p);
   } else {
     if (!attr_set[1]) {
       if ((e = cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
         return e;
       attr_set[1] = true;
     }
-    prefill_kernel<128><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, p);
+    prefill_kernel<128><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, p);
   }
   return cudaGetLastError();
 }

@@ -430,11 +430,13 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
   const int H = h->cfg.num_kv_heads;
   for (size_t i = 0; i < items.size(); ++i)
     it[i] = make_int2(items[i].b, (int)make_item_w1(h->cls[layer * H + items[i].h] != 0, items[i].h, items[i].t));
-  CUtensorMap qmap;
+  CUtensorMap qmap, omap;  // query in, output out: the same [tokens, Hq, D] geometry and tile box
   const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads;
   if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
+                kPrefillTileRows / h->G) ||
+      !make_map(&omap, out, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
                 kPrefillTileRows / h->G)) {
-    h->last_error = "query tensor map encode failed";
+    h->last_error = "query/output tensor map encode failed";
     return SEGKV_ERR_CUDA;
   }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -454,7 +456,7 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
   p.visited = reinterpret_cast<unsigned long long *>(visited);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
-  SEGKV_CUDA(h, "prefill launch", launch_prefill(p, qmap, h->kmap, h->vmap, st));
+  SEGKV_CUDA(h, "prefill launch", launch_prefill(p, qmap, h->kmap, h->vmap, omap, st));
   return SEGKV_OK;
 }
 

@@ -51,11 +51,23 @@ cudaError_t launch_reset(const StorageGeom &g, int num_layers, cudaStream_t st);
 cudaError_t launch_append(const StorageGeom &g, int layer, const void *ws_meta, int nseq, const uint8_t *cls_dev,
                           int total_tokens, const void *k_new, const void *v_new, cudaStream_t st);
 
+// A prefill work item is four int32 words: w0 = sequence index in the call, w1 as above
+// (tile = index of the item's pair of query tiles), w2 = (first key tile << 16) | last key
+// tile of the item's key range, w3 = partial-result slot (-1: the item covers its whole key
+// range and writes out/lse itself; else one chunk of a longer item's key range, whose
+// normalised fp32 O and lse go to slot w3 for the combine kernel).
+// A combine group is four int32 words: w0 = sequence index, w1 as above, w2 = first slot,
+// w3 = number of chunks.
+constexpr int kMaxPartSlots = 320;  // partial-result slots of one prefill call (>= 2 x 148 SMs)
+
 struct PrefillLaunch {
   StorageGeom g;
   int layer, nseq, n_items, tile_pos, grid;
-  const void *ws_meta;  // header + PrefillSeq[nseq] + items
+  const void *ws_meta;  // header + PrefillSeq[nseq] + items (int4) + combine groups (int4)
   int items_off;        // byte offset of the item array inside ws_meta
+  int groups_off, n_groups;
+  float *part_o;        // [slot][2 tiles][D / 4][128 rows] float4: each chunk's O, normalised
+  float *part_lse;      // [slot][2 tiles][128 rows]: each chunk's lse (-inf: no visible key)
   const void *q;
   void *out;
   float *lse;

@@ -76,7 +76,7 @@ struct Smem {
 };
 
 struct Item {
-  int b, h, t, q_first, q_last, lo_min, kt_lo, kt_hi, seq_id, kv_len, q_row;
+  int b, h, t, q_first, q_last, lo_min, kt_lo, kt_hi, seq_id, kv_len, q_row, slot;
   bool global;
 };
 
@@ -94,10 +94,11 @@ struct Bars {
 
 
 // Item = (sequence b, KV head h, tile pair t): positions [q_start + 2 t tp, ...) of the
-// sequence's queries, tp = 128 / G positions per query tile.
-__device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const PrefillSeq *seqs, const int2 *items,
+// sequence's queries, tp = 128 / G positions per query tile, over key tiles [kt_lo, kt_hi]
+// (the item's whole key range, or one chunk of it when slot >= 0).
+__device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const PrefillSeq *seqs, const int4 *items,
                                             int idx) {
-  const int2 w = items[idx];
+  const int4 w = items[idx];
   Item it;
   it.b = w.x;
   const uint32_t w1 = (uint32_t)w.y;
@@ -112,8 +113,9 @@ __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const Prefil
   it.q_last = s.q_start + min((it.t + 1) * pair, s.q_len) - 1;
   it.q_row = s.q_row0 + it.t * pair;
   it.lo_min = it.global ? 0 : max(0, it.q_first - p.g.window + 1);
-  it.kt_lo = it.lo_min / kBN;
-  it.kt_hi = it.q_last / kBN;
+  it.kt_lo = (int)((uint32_t)w.z >> 16);
+  it.kt_hi = w.z & 0xFFFF;
+  it.slot = w.w;
   return it;
 }
 
@@ -121,7 +123,7 @@ __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const Prefil
 template <int D>
 __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUtensorMap &kmap,
                                               const CUtensorMap &vmap, const PrefillLaunch &p, Bars *bar,
-                                              const PrefillSeq *seqs, const int2 *items, uint8_t *q_s, uint8_t *k_s,
+                                              const PrefillSeq *seqs, const int4 *items, uint8_t *q_s, uint8_t *k_s,
                                               uint8_t *v_s, int *sched_next, int lane, int G, int32_t *state,
                                               volatile int *abort_flag) {
   using S = Smem<D>;
@@ -222,7 +224,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
 
 // ---------------------------------------------------------------------------- MMA thread
 template <int D>
-__device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, const PrefillSeq *seqs, const int2 *items,
+__device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, const PrefillSeq *seqs, const int4 *items,
                                          uint8_t *q_s, uint8_t *k_s, uint8_t *v_s, uint32_t tmem, int32_t *state,
                                          volatile int *abort_flag) {
   using S = Smem<D>;
@@ -304,7 +306,7 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
 // ---------------------------------------------------------------------------- softmax warpgroups
 template <int D>
 __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const PrefillLaunch &p, Bars *bar,
-                                             const PrefillSeq *seqs, const int2 *items, uint8_t *o_stage,
+                                             const PrefillSeq *seqs, const int4 *items, uint8_t *o_stage,
                                              uint32_t tmem, int warp, int lane, int G, int32_t *state,
                                              volatile int *abort_flag) {
   using S = Smem<D>;
@@ -408,53 +410,77 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
     // epilogue: the item's last PV into O_t
     if (!warp_wait(&bar->pv_done[tq], (uint32_t)i & 1, abort_flag, state)) break;  // one phase per item
     tc_fence_after();
-    uint32_t o[D];
-#pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(t_o + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[cc * 32]));
-    tmem_ld_wait();
-    tc_fence_before();
-    mbar_arrive(&bar->o_free[tq]);  // O_t is in registers: the next item's first PV may overwrite it
     const float inv_l = (valid && l > 0.f) ? 1.f / l : 0.f;
     const long long orow = (long long)(it.q_row + pos_local) * p.g.hq + it.h * G + g;
-    // a tile whose rows are all real queries goes out through TMA; the last tile of a
-    // sequence may run past it (those rows belong to the next sequence) and is stored row
-    // by row
-    if (it.q_first + (tq + 1) * p.tile_pos - 1 <= it.q_last) {
-      uint8_t *stg = o_stage + tq * Smem<D>::kOStageBytes;
-      const bool leader = (threadIdx.x & 127) == 0;
+    if (it.slot >= 0) {
+      // one chunk of a longer item: O normalised by this chunk's own sum and its lse go to
+      // the chunk's slot (float4 columns, rows contiguous), merged by the combine kernel;
+      // O streams out of TMEM 32 columns at a time
+      float4 *po = reinterpret_cast<float4 *>(p.part_o) + ((long long)it.slot * 2 + tq) * (D / 4) * kTileRows + row;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(t_o + cc * 32, o);
+        tmem_ld_wait();
 #pragma unroll
-      for (int hh = 0; hh < D / 64; ++hh) {
-        uint32_t w[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[hh * 64 + 2 * e]) * inv_l, __uint_as_float(o[hh * 64 + 2 * e + 1]) * inv_l);
-        if (leader) bulk_wait_read_all();  // the previous store has read the buffer
-        named_bar_sync(1 + tq, 128);
-        // row r of the box at r * 128 bytes, 16-byte chunk c at (c ^ (r mod 8)): the
-        // 128-byte swizzle the output tensor map expects
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(stg + row * 128 + ((c ^ (row & 7)) << 4)) =
-              make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-        fence_async_smem();
-        named_bar_sync(1 + tq, 128);
-        if (leader) {
-          tma_store_3d(&omap, stg, hh * 64, it.h * G, it.q_row + tq * p.tile_pos);
-          bulk_commit();
-        }
+        for (int v = 0; v < 8; ++v)
+          po[(cc * 8 + v) * kTileRows] =
+              make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                          __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
       }
-    } else if (valid) {
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
+      tc_fence_before();
+      mbar_arrive(&bar->o_free[tq]);
+      p.part_lse[((long long)it.slot * 2 + tq) * kTileRows + row] =
+          l > 0.f ? (m_used + fast_log2(l)) * 0.69314718055994531f : -INFINITY;
+    } else {
+      uint32_t o[D];
 #pragma unroll
-      for (int v = 0; v < D / 8; ++v)
-        dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l),
-                            pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l),
-                            pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l),
-                            pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(t_o + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[cc * 32]));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bar->o_free[tq]);  // O_t is in registers: the next item's first PV may overwrite it
+      if (it.q_first + (tq + 1) * p.tile_pos - 1 <= it.q_last) {
+        // a tile whose rows are all real queries goes out through TMA; the last tile of a
+        // sequence may run past it (those rows belong to the next sequence) and is stored
+        // row by row
+        uint8_t *stg = o_stage + tq * Smem<D>::kOStageBytes;
+        const bool leader = (threadIdx.x & 127) == 0;
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh) {
+          uint32_t w[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(o[hh * 64 + 2 * e]) * inv_l, __uint_as_float(o[hh * 64 + 2 * e + 1]) * inv_l);
+          if (leader) bulk_wait_read_all();  // the previous store has read the buffer
+          named_bar_sync(1 + tq, 128);
+          // row r of the box at r * 128 bytes, 16-byte chunk c at (c ^ (r mod 8)): the
+          // 128-byte swizzle the output tensor map expects
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4 *>(stg + row * 128 + ((c ^ (row & 7)) << 4)) =
+                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          fence_async_smem();
+          named_bar_sync(1 + tq, 128);
+          if (leader) {
+            tma_store_3d(&omap, stg, hh * 64, it.h * G, it.q_row + tq * p.tile_pos);
+            bulk_commit();
+          }
+        }
+      } else if (valid) {
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
+#pragma unroll
+        for (int v = 0; v < D / 8; ++v)
+          dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
+      }
     }
-    if (valid) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;
+    if (valid && it.slot < 0) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;
     if (p.visited) {
-      unsigned long long cnt = valid ? (unsigned long long)(pq - lo + 1) : 0ull;
+      // visible keys of this row inside the item's key tiles (all of them unless chunked)
+      const int k_lo = max(lo, it.kt_lo * kBN), k_hi = min(pq, it.kt_hi * kBN + kBN - 1);
+      unsigned long long cnt = (valid && k_hi >= k_lo) ? (unsigned long long)(k_hi - k_lo + 1) : 0ull;
       if (G < 32) {
         for (int off = G; off < 32; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
         if (lane < G && cnt) atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + lane], cnt);
@@ -485,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const char *meta = static_cast<const char *>(p.ws_meta);
   int *sched_next = const_cast<int *>(reinterpret_cast<const int *>(meta));
   const PrefillSeq *seqs = reinterpret_cast<const PrefillSeq *>(meta + kHeaderBytes);
-  const int2 *items = reinterpret_cast<const int2 *>(meta + p.items_off);
+  const int4 *items = reinterpret_cast<const int4 *>(meta + p.items_off);
   const int G = p.g.hq / p.g.hkv;
   int32_t *state = p.g.state;
   volatile int *abort_flag = &bar->abort_flag;
@@ -541,6 +567,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Merges the chunks of each split item: lse = log sum_i exp(lse_i), O = sum_i exp(lse_i -
+// lse) O_i (each O_i normalised by its own chunk's sum), bf16 out rounded to nearest even.
+// One CTA per (group, query tile), one thread per row.
+template <int D>
+__global__ void __launch_bounds__(kTileRows) prefill_combine_kernel(const PrefillLaunch p) {
+  const char *meta = static_cast<const char *>(p.ws_meta);
+  const PrefillSeq *seqs = reinterpret_cast<const PrefillSeq *>(meta + kHeaderBytes);
+  const int4 gr = reinterpret_cast<const int4 *>(meta + p.groups_off)[blockIdx.x >> 1];
+  const int tq = blockIdx.x & 1, row = threadIdx.x;
+  const int G = p.g.hq / p.g.hkv, h = item_head((uint32_t)gr.y), tp = item_tile((uint32_t)gr.y);
+  const PrefillSeq s = seqs[gr.x];
+  const int pos_local = tq * p.tile_pos + row / G, g = row % G;
+  if (tp * 2 * p.tile_pos + pos_local >= s.q_len) return;  // past the sequence's last query
+  const long long orow = (long long)(s.q_row0 + tp * 2 * p.tile_pos + pos_local) * p.g.hq + h * G + g;
+  float m = -INFINITY;
+  for (int i = 0; i < gr.w; ++i) m = fmaxf(m, p.part_lse[((long long)(gr.z + i) * 2 + tq) * kTileRows + row]);
+  float wsum = 0.f, w[32];  // the planner cuts an item into at most 32 chunks
+  const int n = min(gr.w, 32);
+  for (int i = 0; i < n; ++i) {
+    const float li = p.part_lse[((long long)(gr.z + i) * 2 + tq) * kTileRows + row];
+    w[i] = li == -INFINITY ? 0.f : expf(li - m);
+    wsum += w[i];
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  const float4 *po = reinterpret_cast<const float4 *>(p.part_o);
+  uint2 *dst = reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
+  for (int v = 0; v < D / 4; ++v) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < n; ++i) {
+      const float4 x = po[(((long long)(gr.z + i) * 2 + tq) * (D / 4) + v) * kTileRows + row];
+      a.x += w[i] * x.x;
+      a.y += w[i] * x.y;
+      a.z += w[i] * x.z;
+      a.w += w[i] * x.w;
+    }
+    dst[v] = make_uint2(pack_bf16x2(a.x * inv, a.y * inv), pack_bf16x2(a.z * inv, a.w * inv));
+  }
+  p.lse[orow] = m + logf(wsum);
+}
+
 }  // namespace
 
 int prefill_smem_bytes(int head_dim) { return head_dim == 64 ? Smem<64>::kBytes : Smem<128>::kBytes; }
@@ -557,6 +623,7 @@ cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, cons
       attr_set[0] = true;
     }
     prefill_kernel<64><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, p);
+    if (p.n_groups > 0) prefill_combine_kernel<64><<<2 * p.n_groups, kTileRows, 0, st>>>(p);
   } else {
     if (!attr_set[1]) {
       if ((e = cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
@@ -564,6 +631,7 @@ cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, cons
       attr_set[1] = true;
     }
     prefill_kernel<128><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, p);
+    if (p.n_groups > 0) prefill_combine_kernel<128><<<2 * p.n_groups, kTileRows, 0, st>>>(p);
   }
   return cudaGetLastError();
 }

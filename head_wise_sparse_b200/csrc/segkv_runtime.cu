@@ -29,6 +29,7 @@ constexpr int kDecodeStageKeys = 64;   // keys of a decode pipeline stage
 constexpr int kMaxSplits = 32;         // most splits one decode head is cut into
 constexpr int kMaxPairs = 8192;        // (sequence, KV head) pairs of one append
 constexpr int kStagingSlots = 4;
+constexpr int kMaxChunks = 32;         // most chunks one prefill item is cut into
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -197,6 +198,14 @@ struct PlanItem {
   int32_t b, h, t, cost;
 };
 
+// One launched work item: a whole item (slot -1) or a chunk [kt_a, kt_b] of its key tiles.
+struct PlanChunk {
+  int32_t b, h, t, kt_a, kt_b, slot;
+};
+struct SplitGroup {
+  int32_t b, h, t, first_slot, n;
+};
+
 // Longest-processing-time-first list: enumerate (b, head, tile), cost = key tiles the
 // tile touches, counting sort by cost descending (stable: ties keep enumeration order).
 void plan_prefill_items(const segkv_t *h, int layer, int nseq, const int32_t *q_start, const int32_t *q_len,
@@ -226,6 +235,83 @@ void plan_prefill_items(const segkv_t *h, int layer, int nseq, const int32_t *q_
   }
   out.assign(items.size(), PlanItem{0, 0, 0, 0});
   for (const PlanItem &it : items) out[start[it.cost]++] = it;
+}
+
+// Key tiles [kt_lo, kt_hi] an item of (sequence b, head k, tile pair t) touches.
+void item_key_range(const segkv_t *h, int layer, int b, int k, int t, const int32_t *q_start, const int32_t *q_len,
+                    int *kt_lo, int *kt_hi) {
+  const int tile_pos = kPrefillItemRows / h->G, W = h->cfg.window;
+  const bool global = h->cls[layer * h->cfg.num_kv_heads + k] != 0;
+  const int q_first = q_start[b] + t * tile_pos;
+  const int q_last = q_start[b] + std::min((t + 1) * tile_pos, q_len[b]) - 1;
+  const int lo = global ? 0 : std::max(0, q_first - W + 1);
+  *kt_lo = lo / kPrefillKeyTile;
+  *kt_hi = q_last / kPrefillKeyTile;
+}
+
+// Cuts items longer than one SM's share of the work into chunks of contiguous key tiles,
+// so that the longest-first schedule can balance: a global head's item can be far longer
+// than total / SMs (for a 4096-query chunk at 128K context about twice as long).  Only
+// when the longest item exceeds the per-SM share; chunks are at least 8 key tiles and at
+// most kMaxPartSlots chunks are made.  The result is again sorted longest first (stable).
+void split_long_items(const segkv_t *h, int layer, const int32_t *q_start, const int32_t *q_len,
+                      const std::vector<PlanItem> &items, int grid, std::vector<PlanChunk> &chunks,
+                      std::vector<SplitGroup> &groups) {
+  long long total = 0;
+  int max_cost = 0;
+  for (const PlanItem &it : items) {
+    total += it.cost;
+    max_cost = std::max(max_cost, it.cost);
+  }
+  const long long fair = (total + grid - 1) / std::max(grid, 1);
+  long long T = max_cost + 1;  // no split
+  if (max_cost > fair) {
+    // at least 8 key tiles a chunk, at most kMaxChunks chunks an item (the combine's limit)
+    T = std::max<long long>({8, (fair + 1) / 2, (max_cost + kMaxChunks - 1) / kMaxChunks});
+    for (;;) {
+      long long slots = 0;
+      for (const PlanItem &it : items)
+        if (it.cost > T) slots += (it.cost + T - 1) / T;
+      if (slots <= kMaxPartSlots) break;
+      T = T + T / 4 + 1;
+    }
+  }
+  chunks.clear();
+  groups.clear();
+  chunks.reserve(items.size() + (max_cost > T ? kMaxPartSlots : 0));
+  if (max_cost <= T) {  // nothing to cut: the list keeps its longest-first order
+    for (const PlanItem &it : items) {
+      int a = 0, z = 0;
+      item_key_range(h, layer, it.b, it.h, it.t, q_start, q_len, &a, &z);
+      chunks.push_back({it.b, it.h, it.t, a, z, -1});
+    }
+    return;
+  }
+  int slot = 0;
+  for (const PlanItem &it : items) {
+    int a = 0, z = 0;
+    item_key_range(h, layer, it.b, it.h, it.t, q_start, q_len, &a, &z);
+    if (it.cost <= T) {
+      chunks.push_back({it.b, it.h, it.t, a, z, -1});
+      continue;
+    }
+    const int n = (int)((it.cost + T - 1) / T);
+    groups.push_back({it.b, it.h, it.t, slot, n});
+    for (int i = 0; i < n; ++i) {
+      const int ca = a + (int)((long long)it.cost * i / n), cz = a + (int)((long long)it.cost * (i + 1) / n) - 1;
+      chunks.push_back({it.b, it.h, it.t, ca, cz, slot++});
+    }
+  }
+  std::stable_sort(chunks.begin(), chunks.end(),
+                   [](const PlanChunk &x, const PlanChunk &y) { return x.kt_b - x.kt_a > y.kt_b - y.kt_a; });
+}
+
+// Prefill workspace: metadata (header, sequences, items, groups), then the partials.
+size_t prefill_meta_bytes(int nseq, size_t n_items, size_t n_groups) {
+  return align_up(align_up(kHeaderBytes + sizeof(PrefillSeq) * nseq, 16) + 16 * n_items + 16 * n_groups, 256);
+}
+size_t prefill_part_bytes(int head_dim) {
+  return (size_t)kMaxPartSlots * 2 * 128 * ((size_t)head_dim + 1) * 4;
 }
 
 }  // namespace
@@ -306,8 +392,9 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
   const size_t H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
   const int tile_pos = kPrefillItemRows / h->G;
   const size_t app = kHeaderBytes + sizeof(AppendSeq) * max_batch + H;
-  const size_t pre = kHeaderBytes + sizeof(PrefillSeq) * max_batch +
-                     8 * H * ((size_t)ceil_div(max_tokens, tile_pos) + max_batch) + 16;
+  const size_t pre = prefill_meta_bytes(max_batch, H * ((size_t)ceil_div(max_tokens, tile_pos) + max_batch) +
+                                                      kMaxPartSlots, kMaxPartSlots) +
+                     prefill_part_bytes((int)D);
   const size_t dec_meta = align_up(kHeaderBytes + sizeof(DecodeSeq) * max_batch + 4 * max_batch * H +
                                        8 * max_batch * H * kMaxSplits + 16,
                                    256);
@@ -410,12 +497,18 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
   if (tq == 0) return SEGKV_OK;
   if (tq > (1LL << 30)) return SEGKV_ERR_UNSUPPORTED;
   if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4)) return SEGKV_ERR_INVALID_ARG;
+  if ((rc = ensure_device_state(h))) return rc;
   std::vector<PlanItem> items;
   plan_prefill_items(h, layer, nseq, q_start_pos, q_len, items);
+  std::vector<PlanChunk> chunks;
+  std::vector<SplitGroup> groups;
+  split_long_items(h, layer, q_start_pos, q_len, items, h->num_sms, chunks, groups);
   const int items_off = (int)align_up(kHeaderBytes + sizeof(PrefillSeq) * nseq, 16);
-  const size_t bytes = items_off + 8 * items.size();
-  if (!ws || !aligned(ws, 256) || ws_bytes < bytes) return SEGKV_ERR_WORKSPACE;
-  if ((rc = ensure_device_state(h))) return rc;
+  const int groups_off = items_off + 16 * (int)chunks.size();
+  const size_t bytes = groups_off + 16 * groups.size();
+  const size_t meta = prefill_meta_bytes(nseq, chunks.size(), groups.size());
+  const size_t need = meta + prefill_part_bytes(h->cfg.head_dim);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEGKV_ERR_WORKSPACE;
   void *host = nullptr;
   if ((rc = staging(h, bytes, &host))) return rc;
   std::memset(host, 0, items_off);
@@ -426,10 +519,18 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
                        h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]], 0, 0, 0};
     row0 += q_len[b];
   }
-  int2 *it = reinterpret_cast<int2 *>(static_cast<char *>(host) + items_off);
+  int4 *it = reinterpret_cast<int4 *>(static_cast<char *>(host) + items_off);
   const int H = h->cfg.num_kv_heads;
-  for (size_t i = 0; i < items.size(); ++i)
-    it[i] = make_int2(items[i].b, (int)make_item_w1(h->cls[layer * H + items[i].h] != 0, items[i].h, items[i].t));
+  for (size_t i = 0; i < chunks.size(); ++i) {
+    const PlanChunk &c = chunks[i];
+    it[i] = make_int4(c.b, (int)make_item_w1(h->cls[layer * H + c.h] != 0, c.h, c.t), (c.kt_a << 16) | c.kt_b,
+                      c.slot);
+  }
+  int4 *gr = reinterpret_cast<int4 *>(static_cast<char *>(host) + groups_off);
+  for (size_t i = 0; i < groups.size(); ++i) {
+    const SplitGroup &g = groups[i];
+    gr[i] = make_int4(g.b, (int)make_item_w1(h->cls[layer * H + g.h] != 0, g.h, g.t), g.first_slot, g.n);
+  }
   CUtensorMap qmap, omap;  // query in, output out: the same [tokens, Hq, D] geometry and tile box
   const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads;
   if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
@@ -445,11 +546,15 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
   p.g = geom(h);
   p.layer = layer;
   p.nseq = nseq;
-  p.n_items = (int)items.size();
+  p.n_items = (int)chunks.size();
   p.tile_pos = kPrefillTileRows / h->G;
-  p.grid = std::min<int>((int)items.size(), h->num_sms);
+  p.grid = std::min<int>((int)chunks.size(), h->num_sms);
   p.ws_meta = ws;
   p.items_off = items_off;
+  p.groups_off = groups_off;
+  p.n_groups = (int)groups.size();
+  p.part_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta);
+  p.part_lse = p.part_o + (size_t)kMaxPartSlots * 2 * 128 * h->cfg.head_dim;
   p.q = q;
   p.out = out;
   p.lse = lse;

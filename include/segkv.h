@@ -98,7 +98,9 @@ int segkv_pages_used(const segkv_t *h);
 
 /* Bytes of device workspace any call with at most max_batch sequences and at most
  * max_tokens packed tokens needs.  Workspace must be 256-byte aligned; calls on the
- * same stream may share one workspace. */
+ * same stream may share one workspace.  It includes a fixed area of 320 x 256 x
+ * (head_dim + 1) x 4 bytes (about 42 MB at head_dim 128) for the partial results of
+ * prefill items cut into key-range chunks (see segkv_prefill_attn). */
 size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens);
 
 /* Empties every sequence: page table <- -1, state <- 0 (device, enqueued), lengths <- 0 (host). */
@@ -132,6 +134,13 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
  * and every one of them must already be appended (q_start_pos + q_len <= seq len).
  * q, out: DEVICE bf16 [sum(q_len), Hq, D] packed in call order; lse: DEVICE fp32
  * [sum(q_len), Hq].  Host arrays: seq_ids, q_start_pos, q_len [nseq].
+ * Scheduling: items (a pair of query tiles of one KV head) run longest first on one
+ * persistent CTA per SM.  When the longest item exceeds the per-SM share of the call's
+ * key tiles (a global head's item against short local ones), such items are cut into
+ * chunks of consecutive key tiles (at least 8 tiles, at most 32 chunks an item); each
+ * chunk writes its normalised fp32 O and lse to the workspace and a combine kernel
+ * merges them (lse = log sum exp of the chunks' lse).  Results do not depend on the
+ * schedule beyond rounding.
  * Errors: INVALID_ARG, RING_TOO_SMALL (a local head's ring dropped a key some query
  * needs), WORKSPACE, CUDA.
  */
@@ -140,7 +149,8 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
                        uint64_t *visited, void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Longest-processing-time-first work list the prefill call would run (host only, no GPU).
+ * Longest-processing-time-first work list of the prefill call, before any item is cut into
+ * key chunks (host only, no GPU).
  * Item = (b, kv head, query tile, cost); a query tile holds tile_pos = 256 / G consecutive
  * positions of all G query heads of the KV head; cost = number of key_tile-aligned key
  * tiles meeting [lo, q_last] (lo = 0 global, max(0, q_first - W + 1) local); order: cost

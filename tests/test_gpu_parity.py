@@ -96,6 +96,16 @@ def test_mistral_shape_scaled_length(torch_cuda):
     check_against_oracle(w, 0, q, out, lse, vis, ids, qs, ql)
 
 
+def test_long_items_cut_into_key_chunks(torch_cuda):
+    # one global KV head under 8 query heads: 128 items of 1..32 key tiles against a per-SM
+    # share of about 15, so the longer items run as several key-range chunks merged by the
+    # combine kernel; a local head beside it keeps whole items
+    w = Workload(320, "chunks", 1, 16, 2, 128, 64, 700, 64, (Seq(0, 4096, 0, 4096),), ((1, 0),))
+    kv, q, out, lse, vis = run_prefill_case(torch_cuda, w)
+    ids, qs, ql = step_queries(w)
+    check_against_oracle(w, 0, q, out, lse, vis, ids, qs, ql)
+
+
 def test_chunked_prefill_at_offset_with_ring(torch_cuda):
     w = wl.CONFIGS["mha_chunked_prefill_128k"].scaled(
         seqs=(Seq(6000, 1000, 6000, 7000),), ring_pages=-(-(4096 + 1000 - 1) // 64) + 1)

@@ -366,14 +366,15 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
       const bool rescale = grow && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, rescale)) {
         const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.0f;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(t_o + cc * 32, o);
+        // 16 columns at a time: the whole S row is live here
+#pragma unroll 1
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t o[16];
+          tmem_ld16(t_o + cc * 16, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(t_o + cc * 32, o);
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(t_o + cc * 16, o);
         }
         l *= alpha;
       }
@@ -381,13 +382,14 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      // P in two halves of 64 keys; the MMA thread starts each half's PV as it lands
+      // P in two halves of 64 keys (each stored as two quarters of 32 keys); the MMA thread
+      // starts each half's PV as it lands
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t pk[32];
+      for (int qq = 0; qq < 4; ++qq) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float2 x = ffma2(make_float2(s[cc * 64 + 2 * e], s[cc * 64 + 2 * e + 1]), c2, nm2);
+        for (int e = 0; e < 16; ++e) {
+          const float2 x = ffma2(make_float2(s[qq * 32 + 2 * e], s[qq * 32 + 2 * e + 1]), c2, nm2);
           float2 pe;
           if (kEmuEvery > 0 && e % (kEmuEvery > 0 ? kEmuEvery : 1) == kEmuEvery - 1)
             pe = exp2_fma2(x);
@@ -396,10 +398,12 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
           acc[e & 3] = fadd2(acc[e & 3], pe);
           pk[e] = pack_bf16x2(pe.x, pe.y);
         }
-        tmem_st32(t_s + cc * 32, pk);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(cc == 0 ? &bar->p_lo[tq] : &bar->p_hi[tq]);
+        tmem_st16(t_s + qq * 16, pk);
+        if (qq & 1) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(qq == 1 ? &bar->p_lo[tq] : &bar->p_hi[tq]);
+        }
       }
       const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
       const float2 a = fadd2(a01, a23);
@@ -433,12 +437,20 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
       p.part_lse[((long long)it.slot * 2 + tq) * kTileRows + row] =
           l > 0.f ? (m_used + fast_log2(l)) * 0.69314718055994531f : -INFINITY;
     } else {
-      uint32_t o[D];
+      // O leaves TMEM 64 columns at a time, normalised and packed to bf16 on the way
+      uint32_t w[D / 2];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(t_o + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[cc * 32]));
-      tmem_ld_wait();
+      for (int hh = 0; hh < D / 64; ++hh) {
+        uint32_t o[64];
+        tmem_ld32(t_o + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+        tmem_ld32(t_o + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          w[hh * 32 + e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+      }
       tc_fence_before();
-      mbar_arrive(&bar->o_free[tq]);  // O_t is in registers: the next item's first PV may overwrite it
+      mbar_arrive(&bar->o_free[tq]);  // O_t is read: the next item's first PV may overwrite it
       if (it.q_first + (tq + 1) * p.tile_pos - 1 <= it.q_last) {
         // a tile whose rows are all real queries goes out through TMA; the last tile of a
         // sequence may run past it (those rows belong to the next sequence) and is stored
@@ -447,10 +459,6 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
         const bool leader = (threadIdx.x & 127) == 0;
 #pragma unroll
         for (int hh = 0; hh < D / 64; ++hh) {
-          uint32_t w[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(o[hh * 64 + 2 * e]) * inv_l, __uint_as_float(o[hh * 64 + 2 * e + 1]) * inv_l);
           if (leader) bulk_wait_read_all();  // the previous store has read the buffer
           named_bar_sync(1 + tq, 128);
           // row r of the box at r * 128 bytes, 16-byte chunk c at (c ^ (r mod 8)): the
@@ -458,7 +466,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             *reinterpret_cast<uint4 *>(stg + row * 128 + ((c ^ (row & 7)) << 4)) =
-                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                make_uint4(w[hh * 32 + 4 * c], w[hh * 32 + 4 * c + 1], w[hh * 32 + 4 * c + 2], w[hh * 32 + 4 * c + 3]);
           fence_async_smem();
           named_bar_sync(1 + tq, 128);
           if (leader) {
@@ -469,11 +477,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
       } else if (valid) {
         uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
 #pragma unroll
-        for (int v = 0; v < D / 8; ++v)
-          dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l),
-                              pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l),
-                              pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l),
-                              pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
+        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
       }
     }
     if (valid && it.slot < 0) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;

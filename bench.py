@@ -381,7 +381,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": PREFILL, "seq_len": L, "q_heads": w.hq, "kv_heads": w.hkv, "head_dim": w.d,
                    "page_size": w.page, "window": w.window, "global_kv_heads": int(sum(w.classes[0])),
-                   "visible_pairs": visible_pairs(w), "step": "reset + append (page build, scatter) + prefill",
+                   "visible_pairs": visible_pairs(w), "step": "reset + append (page ids + scatter) + prefill",
                    "l2": "flushed between timed steps (256 MiB write, outside the events)",
                    "parallelism": f"replicas x{world}"},
         "prefill_kernel_ms": t_pre, "append_ms": max_over_ranks(sum(app_ms) / args.steps),
@@ -390,7 +390,7 @@ def main():
                      "peak_source": f"{pk_src} bf16 burst",
                      "kernel": "prefill_kernel<128> (events around segkv_prefill_attn: metadata upload + kernel)"},
         "e2e": e2e,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clocks,
     }
     if decode is not None:
@@ -469,11 +469,11 @@ def bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk):
     res = {
         "workload": DECODE, "metric": "decode KV GB/s", "value": world * per_step / (t_step * 1e-3) / 1e9,
         "unit": "GB/s", "ms_per_step": t_step, "decode_kernel_ms": t_dec, "steps": steps,
-        "kv_bytes_per_step": per_step, "step": "append 1 token/seq (page build + scatter) + split-K decode + combine",
+        "kv_bytes_per_step": per_step, "step": "append 1 token/seq (page ids + scatter) + split-K decode + combine",
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic("decode_64x32k.md", DECODE_SOURCES),
                      "kernel": "decode_split_kernel<128> + lse_combine (events around segkv_decode_attn)"},
-        "gpu_launches": 4 * steps, "data": "synthetic (seeded torch generator on the device)",
+        "gpu_launches": 3 * steps, "data": "synthetic (seeded torch generator on the device)",
     }
     del kv
     torch.cuda.empty_cache()

@@ -49,7 +49,8 @@ struct StorageGeom {  // what every kernel needs to resolve a logical position t
 cudaError_t launch_reset(const StorageGeom &g, int num_layers, cudaStream_t st);
 
 cudaError_t launch_append(const StorageGeom &g, int layer, const void *ws_meta, int nseq, const uint8_t *cls_dev,
-                          int total_tokens, const void *k_new, const void *v_new, cudaStream_t st);
+                          const int32_t *pair_off_dev, int cursor0, int new_pages, int total_tokens,
+                          const void *k_new, const void *v_new, cudaStream_t st);
 
 // A prefill work item is four int32 words: w0 = sequence index in the call, w1 as above
 // (tile = index of the item's pair of query tiles), w2 = (first key tile << 16) | last key

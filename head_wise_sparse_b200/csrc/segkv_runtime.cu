@@ -27,7 +27,6 @@ constexpr int kPrefillItemRows = 256;  // rows of one prefill work item (two que
 constexpr int kPrefillKeyTile = 128;   // keys of a prefill key tile
 constexpr int kDecodeStageKeys = 64;   // keys of a decode pipeline stage
 constexpr int kMaxSplits = 32;         // most splits one decode head is cut into
-constexpr int kMaxPairs = 8192;        // (sequence, KV head) pairs of one append
 constexpr int kStagingSlots = 4;
 constexpr int kMaxChunks = 32;         // most chunks one prefill item is cut into
 
@@ -391,7 +390,7 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
   if (!h || max_batch < 1 || max_tokens < 0) return 0;
   const size_t H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
   const int tile_pos = kPrefillItemRows / h->G;
-  const size_t app = kHeaderBytes + sizeof(AppendSeq) * max_batch + H;
+  const size_t app = kHeaderBytes + sizeof(AppendSeq) * max_batch + align_up(H, 4) + 4 * H * max_batch;
   const size_t pre = prefill_meta_bytes(max_batch, H * ((size_t)ceil_div(max_tokens, tile_pos) + max_batch) +
                                                       kMaxPartSlots, kMaxPartSlots) +
                      prefill_part_bytes((int)D);
@@ -419,8 +418,8 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
   if (rc) return rc;
   if (!start_pos || !num_new) return SEGKV_ERR_INVALID_ARG;
   const int H = h->cfg.num_kv_heads;
-  if ((long long)nseq * H > kMaxPairs) return SEGKV_ERR_UNSUPPORTED;
   long long total = 0, new_pages = 0;
+  std::vector<int32_t> pair_off((size_t)nseq * H);  // pages allocated for earlier (sequence, head) pairs
   for (int b = 0; b < nseq; ++b) {
     const int s = seq_ids[b];
     const int cur = h->len[(size_t)layer * h->cfg.max_seqs + s];
@@ -429,15 +428,19 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
     total += num_new[b];
     for (int k = 0; k < H; ++k) {
       const bool global = h->cls[layer * H + k] != 0;
+      pair_off[(size_t)b * H + k] = (int32_t)new_pages;
       new_pages += held_pages(h, global, cur + num_new[b]) - held_pages(h, global, cur);
     }
   }
   if (total > (1LL << 30)) return SEGKV_ERR_UNSUPPORTED;
   if (total > 0 && (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16))) return SEGKV_ERR_INVALID_ARG;
   if (h->pages_used + new_pages > h->cfg.num_pages) return SEGKV_ERR_OUT_OF_PAGES;
-  const size_t bytes = kHeaderBytes + sizeof(AppendSeq) * nseq + H;
+  const size_t cls_off = kHeaderBytes + sizeof(AppendSeq) * nseq;
+  const size_t off_off = cls_off + align_up(H, 4);
+  const size_t bytes = off_off + 4 * (size_t)H * nseq;
   if (!ws || !aligned(ws, 256) || ws_bytes < bytes) return SEGKV_ERR_WORKSPACE;
   if ((rc = ensure_device_state(h))) return rc;
+  if (total == 0) return SEGKV_OK;
   void *host = nullptr;
   if ((rc = staging(h, bytes, &host))) return rc;
   std::memset(host, 0, kHeaderBytes);
@@ -447,12 +450,15 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
     as[b] = AppendSeq{seq_ids[b], start_pos[b], num_new[b], tok};
     tok += num_new[b];
   }
-  uint8_t *cls = reinterpret_cast<uint8_t *>(as + nseq);
-  std::memcpy(cls, &h->cls[(size_t)layer * H], H);
+  std::memcpy(static_cast<char *>(host) + cls_off, &h->cls[(size_t)layer * H], H);
+  std::memcpy(static_cast<char *>(host) + off_off, pair_off.data(), 4 * (size_t)H * nseq);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = upload(h, ws, bytes, st))) return rc;
-  const uint8_t *cls_dev = static_cast<const uint8_t *>(ws) + kHeaderBytes + sizeof(AppendSeq) * nseq;
-  SEGKV_CUDA(h, "append launch", launch_append(geom(h), layer, ws, nseq, cls_dev, (int)total, k_new, v_new, st));
+  const uint8_t *cls_dev = static_cast<const uint8_t *>(ws) + cls_off;
+  const int32_t *off_dev = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + off_off);
+  SEGKV_CUDA(h, "append launch",
+             launch_append(geom(h), layer, ws, nseq, cls_dev, off_dev, (int)h->pages_used, (int)new_pages, (int)total,
+                           k_new, v_new, st));
   for (int b = 0; b < nseq; ++b) h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] += num_new[b];
   h->pages_used += new_pages;
   return SEGKV_OK;

@@ -367,7 +367,28 @@ def main():
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
     e2e = {"value": world * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e}
-    del kv, flush
+    # ------------------------------------------------------------------ query relocation
+    # segkv_relocate_q on the same workload's queries (local heads turned by -delta, the
+    # global head copied): HBM-bound, one read and one write of every query element.
+    q_rel = torch.empty_like(q_d)
+    shift = torch.full((L,), 100000, dtype=torch.int32, device=dev)
+    for _ in range(args.warmup):
+        kv.relocate_q(0, q_d, shift, out=q_rel)
+    evr = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(args.steps, 50))]
+    for e in evr:
+        flush.fill_(1)
+        e[0].record(stream)
+        kv.relocate_q(0, q_d, shift, out=q_rel)
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    t_rel = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evr) / len(evr))
+    rel_bytes = 2 * q_d.numel() * 2
+    relocate = {"metric": "query relocation GB/s", "value": world * rel_bytes / (t_rel * 1e-3) / 1e9, "unit": "GB/s",
+                "ms_per_call": t_rel, "bytes_per_call": rel_bytes,
+                "roofline": {"bound": "hbm", "achieved": rel_bytes / (t_rel * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": rel_bytes / (t_rel * 1e-3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                             "kernel": "relocate_q_kernel (events around segkv_relocate_q)"}}
+    del kv, flush, q_rel
     torch.cuda.empty_cache()
 
     # ------------------------------------------------------------------ decode workload
@@ -393,6 +414,7 @@ def main():
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
     }
+    line["relocate"] = relocate
     if decode is not None:
         line["decode"] = decode
     if rank == 0 and world == 1 and not args.no_cpu:

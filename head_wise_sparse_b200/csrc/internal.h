@@ -94,4 +94,14 @@ struct DecodeLaunch {
 cudaError_t launch_decode(const DecodeLaunch &p, const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t st);
 int decode_smem_bytes(int head_dim);
 
+struct RelocateLaunch {
+  const int32_t *shift;  // DEVICE [n_tokens]: the position offset of each packed token
+  const void *q_in;
+  void *q_out;
+  int hq, hkv, head_dim, interleaved;
+  double log2_base;
+  uint32_t cls_bits[32];  // class of KV heads 0..1023: bit set = global (passes unchanged)
+};
+cudaError_t launch_relocate_q(const RelocateLaunch &p, int n_tokens, cudaStream_t st);
+
 }  // namespace skv

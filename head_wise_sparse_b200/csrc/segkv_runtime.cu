@@ -659,6 +659,33 @@ int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
   return SEGKV_OK;
 }
 
+int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, const void *q_in, void *q_out,
+                     float theta_base, int interleaved, void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= h->cfg.num_layers || n_tokens < 0 || !(theta_base > 1.0f) ||
+      (interleaved != 0 && interleaved != 1))
+    return SEGKV_ERR_INVALID_ARG;
+  if (n_tokens == 0) return SEGKV_OK;
+  if (!shift || !q_in || !q_out || !aligned(shift, 4) || !aligned(q_in, 16) || !aligned(q_out, 16))
+    return SEGKV_ERR_INVALID_ARG;
+  const int H = h->cfg.num_kv_heads;
+  if (H > 1024 || n_tokens > (1 << 30)) return SEGKV_ERR_UNSUPPORTED;
+  RelocateLaunch p;
+  p.shift = shift;
+  p.q_in = q_in;
+  p.q_out = q_out;
+  p.hq = h->cfg.num_q_heads;
+  p.hkv = H;
+  p.head_dim = h->cfg.head_dim;
+  p.interleaved = interleaved;
+  p.log2_base = std::log2((double)theta_base);
+  std::memset(p.cls_bits, 0, sizeof(p.cls_bits));
+  for (int k = 0; k < H; ++k)
+    if (h->cls[(size_t)layer * H + k]) p.cls_bits[k >> 5] |= 1u << (k & 31);
+  SEGKV_CUDA(h, "relocate launch", launch_relocate_q(p, n_tokens, static_cast<cudaStream_t>(stream)));
+  return SEGKV_OK;
+}
+
 int segkv_device_status(segkv_t *h, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -25,7 +25,7 @@ EXPORTS = [
     "segkv_create", "segkv_destroy", "segkv_ring_pages", "segkv_max_lp", "segkv_seq_len", "segkv_pages_used",
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
     "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
-    "segkv_decode_attn_noalloc",
+    "segkv_decode_attn_noalloc", "segkv_relocate_q",
 ]
 
 
@@ -73,6 +73,7 @@ def lib():
                                          ctypes.POINTER(I)]
         L.segkv_decode_attn.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P, SZ, P]
         L.segkv_decode_attn_noalloc.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P]
+        L.segkv_relocate_q.argtypes = [P, I, I, P, P, P, F, I, P]
         L.segkv_device_status.argtypes = [P, P]
         L.segkv_last_error.argtypes = [P]
         L.segkv_last_error.restype = ctypes.c_char_p
@@ -182,6 +183,10 @@ class Handle:
                                                int(num_splits), _dptr(out), _dptr(lse), _dptr(visited),
                                                _stream(stream))
 
+    def relocate_q(self, layer, n_tokens, shift, q_in, q_out, theta_base, interleaved, stream=None) -> int:
+        return lib().segkv_relocate_q(self.h, layer, int(n_tokens), _dptr(shift), _dptr(q_in), _dptr(q_out),
+                                      float(theta_base), int(interleaved), _stream(stream))
+
     def plan_prefill(self, layer, q_start, q_len):
         """Longest-processing-time-first list as int32 rows (seq index, KV head, tile, cost)."""
         qs, ql = _i32(q_start), _i32(q_len)
@@ -263,6 +268,15 @@ class SegKV:
         _check(self.handle.decode(layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, self.ws,
                                   self.ws_bytes), "segkv_decode_attn", self.handle.h)
         return out, lse
+
+    def relocate_q(self, layer: int, q, shift, *, out=None, theta_base: float = 10000.0, interleaved: bool = False):
+        """segkv_relocate_q: local heads' queries turned by the rotary angle of position -shift
+        (shift: int32 per packed token, on the device); ``out`` may be ``q`` (in place)."""
+        t = self.torch
+        out = out if out is not None else t.empty_like(q)
+        _check(self.handle.relocate_q(layer, q.shape[0], shift, q, out, theta_base, interleaved), "segkv_relocate_q",
+               self.handle.h)
+        return out
 
     def device_status(self) -> int:
         return self.handle.device_status()

@@ -192,6 +192,26 @@ int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const int32_t *se
                               const void *q, float softmax_scale, int num_splits, void *out, float *lse,
                               uint64_t *visited, void *stream);
 
+/*
+ * Query relocation for position-independent reuse of local-head KV ("RedKnot-MLA: Multi-
+ * Head Offline-Online Reuse for DeepSeek-V4 Long-Context Serving", Summary: documents are
+ * prefilled offline at canonical position zero; at serving time the queries are rotated by
+ * the negative position offset).  For every packed token t, the query heads of `layer`'s
+ * local KV heads are turned by the rotary angle of position -shift[t]: dimension pairs
+ * (i, i + D/2) (interleaved = 0) or (2i, 2i + 1) (interleaved = 1) rotate by
+ * -shift[t] * theta_base^(-2i/D).  A query rotated to its true position p and relocated by
+ * delta then scores against a key stored at canonical position j as against that key at
+ * j + delta (rotary scores depend only on position differences).  Query heads of global
+ * KV heads are copied unchanged.
+ *   q_in, q_out: DEVICE bf16 [n_tokens, Hq, D] (the same pointer relocates in place);
+ *   shift: DEVICE int32 [n_tokens].  Angles are formed and reduced modulo 2 pi in fp64,
+ *   the rotation is done in fp32 and rounded to bf16 (nearest even).
+ * Errors: INVALID_ARG (pointers, alignment, theta_base <= 1, interleaved not 0/1),
+ * UNSUPPORTED (more than 1024 KV heads), CUDA.
+ */
+int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, const void *q_in, void *q_out,
+                     float theta_base, int interleaved, void *stream);
+
 /* Synchronizes `stream`, reads the device error word, clears it and returns it
  * (SEGKV_OK, SEGKV_ERR_DEVICE_BOUNDS or SEGKV_ERR_DEVICE_TIMEOUT), or SEGKV_ERR_CUDA. */
 int segkv_device_status(segkv_t *h, void *stream);

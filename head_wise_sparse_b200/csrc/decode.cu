@@ -1,5 +1,5 @@
 // decode.cu -- split-K decode over per-head paged KV storage plus a log-sum-exp combine
-// (north star subsystem (3)).
+// (one query token per sequence).
 //
 // One query token per sequence.  A work item is (sequence, KV head, split): a run of
 // consecutive logical pages of that head's visible range.  The item's G query heads

@@ -1,6 +1,6 @@
 // prefill_sm100.cu -- causal variable-length prefill over per-head paged KV storage,
 // tcgen05 tensor cores with TMEM accumulators, TMA page loads, persistent LPT scheduling
-// (north star subsystems (2) and (4)).
+// (one CTA per SM working through a longest-first list of items).
 //
 // What it computes (zhichai.net news item "What Happened", item 3): for every query row of
 // every head, attention over exactly the keys that head keeps, with the head's visibility

@@ -1,5 +1,4 @@
-// rope.cu -- query relocation for position-independent reuse of local-head KV (survey row
-// "next": RoPE relocation).
+// rope.cu -- query relocation for position-independent reuse of local-head KV.
 //
 // What it computes ("RedKnot-MLA: Multi-Head Offline-Online Reuse for DeepSeek-V4 Long-
 // Context Serving", Summary): documents are prefilled offline at canonical position zero,

@@ -1,4 +1,4 @@
-// storage.cu -- per-head page-table builder and KV append/scatter (north star subsystem (1)).
+// storage.cu -- per-head page tables and the KV append/scatter.
 //
 // The storage itself follows the pages' "per-(layer, head) segmented paged KV storage that
 // physically stores only the tokens each head actually needs" (zhichai.net news item,

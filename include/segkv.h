@@ -108,8 +108,9 @@ int segkv_reset(segkv_t *h, void *stream);
 
 /*
  * Appends tokens [start_pos[b], start_pos[b] + num_new[b]) of sequence seq_ids[b] to every
- * KV head of `layer` (north star subsystem (1): per-head page-table builder and KV
- * append/scatter).  start_pos[b] must equal segkv_seq_len(h, layer, seq_ids[b]); seq ids
+ * KV head of `layer`: the per-head page tables grow and the K/V rows are scattered into the
+ * pages (zhichai.net news item "What Happened", item 3: per-(layer, head) segmented paged
+ * storage).  start_pos[b] must equal segkv_seq_len(h, layer, seq_ids[b]); seq ids
  * in one call are distinct.  k_new / v_new: DEVICE bf16 [sum(num_new), Hkv, D],
  * sequences packed in call order.
  *   Page rule: every unallocated slot touched takes the next id of the free list, in the
@@ -126,8 +127,9 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
                  void *stream);
 
 /*
- * Causal variable-length prefill over the segmented storage (north star subsystems (2)
- * and (4)): for every query row and its query head,
+ * Causal variable-length prefill over the segmented storage (zhichai.net news item "What
+ * Happened", item 3: one fused variable-length attention pass over every head's own
+ * pages): for every query row and its query head,
  *   out = sum_visible softmax(scale * q.k) v   (bf16, RNE),  lse (fp32, natural log),
  *   visited[b, hq] += number of visible (q,k) pairs (u64, may be NULL).
  * Queries of sequence seq_ids[b] sit at positions [q_start_pos[b], q_start_pos[b] + q_len[b])
@@ -162,7 +164,7 @@ int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_s
 
 /*
  * Decode: one query per sequence at position q_pos[b] (already appended), split-K over
- * the head's visible pages plus a log-sum-exp combine (north star subsystem (3)).
+ * the head's visible pages plus a log-sum-exp combine.
  * q, out: DEVICE bf16 [nseq, Hq, D]; lse DEVICE fp32 [nseq, Hq]; visited as for prefill.
  * num_splits: 0 = automatic, else the largest number of splits any head is cut into.
  */

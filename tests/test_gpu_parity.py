@@ -1,6 +1,6 @@
 """CUDA path against the fp64 oracle, through the C ABI (needs a B200).
 
-Tolerances (the benchmark spec): |out - ref| <= 8e-3 + 1e-2 |ref| elementwise on bf16 outputs,
+Tolerances: |out - ref| <= 8e-3 + 1e-2 |ref| elementwise on bf16 outputs,
 |lse - ref| <= 1e-3; page tables, cursor and visited-pair counts bit-exact.
 """
 import numpy as np

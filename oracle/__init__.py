@@ -48,6 +48,7 @@ def _load():
         lib.orc_cursor.argtypes = [P]
         lib.orc_seq_len.argtypes = [P, I, I]
         lib.orc_append.argtypes = [P, I, I, P, P, P, P, P]
+        lib.orc_fork.argtypes = [P, I, I]
         lib.orc_attention.argtypes = [P, I, I, P, P, P, P, D, P, I64, P, P, P, I]
         lib.orc_lpt_items.restype = I64
         lib.orc_lpt_items.argtypes = [I, P, P, I, P, I, I, I, P, I64]
@@ -121,6 +122,12 @@ class Oracle:
         rc = self.lib.orc_append(self.h, layer, len(s), _ptr(s), _ptr(st), _ptr(c), _ptr(k), _ptr(v))
         if rc:
             raise OracleError(f"orc_append failed with {rc}")
+
+    def fork(self, src: int, dst: int) -> None:
+        """The empty sequence dst takes src's pages (shared) and length in every layer."""
+        rc = self.lib.orc_fork(self.h, src, dst)
+        if rc != ORC_OK:
+            raise OracleError(f"orc_fork failed: {rc}")
 
     def attention(self, layer: int, seq_ids: Sequence[int], q_start: Sequence[int], q_len: Sequence[int],
                   q: np.ndarray, scale: Optional[float] = None, rows: Optional[np.ndarray] = None,

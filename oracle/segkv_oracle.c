@@ -19,10 +19,15 @@
  *   visibility of a query at position p:  global  k <= p;   local  p - W < k <= p;
  *   query head h reads KV head h / G (G = Hq / Hkv, contiguous groups);
  *   lse = natural log of the sum of exp(scale * q.k) over visible keys;
- *   page allocation: every unallocated slot touched by an append takes the next id of the
- *   caller's free list, in the order (sequence in call order, KV head ascending, logical
- *   page ascending); a global head maps logical page lp to slot lp, a local head to slot
- *   lp mod R and keeps only the last R logical pages ending at the call's last token.
+ *   page allocation: every slot touched by an append that is unallocated, or whose page is
+ *   shared with another sequence, takes the next id of the caller's free list, in the
+ *   order (sequence in call order, KV head ascending, logical page ascending); a shared
+ *   page's content is copied into the new page first (copy on write); a global head maps
+ *   logical page lp to slot lp, a local head to slot lp mod R and keeps only the last R
+ *   logical pages ending at the call's last token;
+ *   fork (hysenlabs.com write-up, "Experimental Features and Current Limitations": a shared
+ *   KV manager with forks and copy-on-write append): an empty sequence takes a copy of
+ *   another's page-table rows in every layer and its length; the pages become shared.
  *
  * Arithmetic: bf16 inputs are widened exactly to double; everything after that is fp64;
  * exp/log are the host libm's.  Outputs are never rounded.
@@ -49,12 +54,16 @@ typedef struct {
   int32_t cursor;
   int32_t *pt;   /* page table [layers][max_seqs][hkv][max_lp], -1 = unallocated */
   int32_t *len;  /* tokens appended so far [layers][max_seqs] */
-  int64_t *tag;  /* per physical page: which (layer, seq, head, logical page) it holds */
+  int64_t *tag;  /* per physical page: which (layer, head, logical page) it holds */
+  int32_t *ref;  /* per physical page: page-table slots pointing at it */
   uint16_t *kpool, *vpool; /* [num_pages][page][d] bf16 bits */
 } orc_t;
 
+/* A page holds one logical page of one (layer, head); sequences that share it (after a
+ * fork) share that content, so the tag leaves the sequence out. */
 static int64_t make_tag(const orc_t *o, int layer, int seq, int head, int lp) {
-  return (((int64_t)layer * o->max_seqs + seq) * o->hkv + head) * (int64_t)o->max_lp + lp;
+  (void)seq;
+  return ((int64_t)layer * o->hkv + head) * (int64_t)o->max_lp + lp;
 }
 
 static double bf16_to_double(uint16_t b) {
@@ -83,6 +92,7 @@ orc_t *orc_create(int layers, int hq, int hkv, int d, int page, int window, int 
   o->len = (int32_t *)calloc((size_t)layers * max_seqs, sizeof(int32_t));
   o->tag = (int64_t *)malloc(sizeof(int64_t) * (size_t)num_pages);
   for (int i = 0; i < num_pages; ++i) o->tag[i] = -1;
+  o->ref = (int32_t *)calloc((size_t)num_pages, sizeof(int32_t));
   o->kpool = (uint16_t *)calloc((size_t)num_pages * page * d, sizeof(uint16_t));
   o->vpool = (uint16_t *)calloc((size_t)num_pages * page * d, sizeof(uint16_t));
   return o;
@@ -90,7 +100,7 @@ orc_t *orc_create(int layers, int hq, int hkv, int d, int page, int window, int 
 
 void orc_destroy(orc_t *o) {
   if (!o) return;
-  free(o->cls); free(o->free_list); free(o->pt); free(o->len); free(o->tag);
+  free(o->cls); free(o->free_list); free(o->pt); free(o->len); free(o->tag); free(o->ref);
   free(o->kpool); free(o->vpool); free(o);
 }
 
@@ -136,9 +146,18 @@ int orc_append(orc_t *o, int layer, int nseq, const int32_t *seq_ids, const int3
       int32_t *row = pt_row(o, layer, s, h);
       for (int lp = lp0; lp <= lp1; ++lp) {
         int slot = slot_of(o, global, lp);
-        if (row[slot] < 0) {
+        const int32_t old = row[slot];
+        if (old < 0 || o->ref[old] > 1) {
           if (o->cursor >= o->num_pages) return ORC_ERR_OUT_OF_PAGES;
-          row[slot] = o->free_list[o->cursor++];
+          const int32_t fresh = o->free_list[o->cursor++];
+          if (old >= 0) { /* copy on write: the other sequences keep the old page */
+            const size_t bytes = sizeof(uint16_t) * (size_t)P * D;
+            memcpy(o->kpool + (size_t)fresh * P * D, o->kpool + (size_t)old * P * D, bytes);
+            memcpy(o->vpool + (size_t)fresh * P * D, o->vpool + (size_t)old * P * D, bytes);
+            o->ref[old]--;
+          }
+          row[slot] = fresh;
+          o->ref[fresh] = 1;
         }
         o->tag[row[slot]] = make_tag(o, layer, s, h, lp);
       }
@@ -161,6 +180,26 @@ int orc_append(orc_t *o, int layer, int nseq, const int32_t *seq_ids, const int3
       }
     }
     o->len[(size_t)layer * o->max_seqs + s] = count[b] > 0 ? last + 1 : first;
+  }
+  return ORC_OK;
+}
+
+/* Fork: the empty sequence dst takes src's page-table rows and length in every layer; every
+ * page it now points at gains a reference. */
+int orc_fork(orc_t *o, int src, int dst) {
+  if (src < 0 || dst < 0 || src >= o->max_seqs || dst >= o->max_seqs || src == dst) return ORC_ERR_ARG;
+  for (int l = 0; l < o->layers; ++l)
+    if (o->len[(size_t)l * o->max_seqs + dst] != 0) return ORC_ERR_ARG;
+  for (int l = 0; l < o->layers; ++l) {
+    for (int h = 0; h < o->hkv; ++h) {
+      const int32_t *a = pt_row(o, l, src, h);
+      int32_t *b = pt_row(o, l, dst, h);
+      for (int i = 0; i < o->max_lp; ++i) {
+        b[i] = a[i];
+        if (a[i] >= 0) o->ref[a[i]]++;
+      }
+    }
+    o->len[(size_t)l * o->max_seqs + dst] = o->len[(size_t)l * o->max_seqs + src];
   }
   return ORC_OK;
 }

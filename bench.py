@@ -415,6 +415,7 @@ def main():
         "clocks": clocks,
     }
     line["relocate"] = relocate
+    line["fork"] = bench_fork(args, torch, dev, stream, max_over_ranks, world, pk)
     if decode is not None:
         line["decode"] = decode
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -425,6 +426,52 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def bench_fork(args, torch, dev, stream, max_over_ranks, world, pk):
+    """Copy on write after a fork: 64 sequences of 1000 tokens (Mistral-shaped heads) are
+    forked into 64 empty slots; the timed call appends one token to every fork, so each of
+    the 8 heads of each fork first copies its shared, partly filled last page (the rows
+    before the new token) into a fresh page.  Bytes: the copied rows plus the new rows."""
+    from head_wise_sparse_b200.segkv import SegKV
+
+    w = wl.CONFIGS[PREFILL]
+    B, ctx, P = 64, 1000, w.page
+    n_pages = 2 * B * w.hkv * (ctx // P + 2) + 64
+    free = np.random.default_rng(7).permutation(n_pages).astype(np.int32)
+    kv = SegKV(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=P, window=w.window,
+               head_class=w.class_array(), num_pages=n_pages, free_list=free, max_seqs=2 * B, max_seq_len=ctx + 8,
+               ring_pages=-(-(ctx + 8) // P), max_chunk=ctx, ws_batch=B, ws_tokens=B * ctx, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    k = torch.randn((B * ctx, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    k1 = torch.randn((B, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    src, dst = list(range(B)), list(range(B, 2 * B))
+    times = []
+    for it in range(args.warmup + 10):
+        kv.reset()
+        kv.append(0, src, [0] * B, [ctx] * B, k, k)
+        for a, b in zip(src, dst):
+            kv.fork(a, b)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kv.append(0, dst, [ctx] * B, [1] * B, k1, k1)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the fork benchmark")
+    t = max_over_ranks(statistics.median(times))
+    moved = B * w.hkv * ((ctx % P) + 1) * w.d * 2 * 2 * 2  # K and V: copied rows read + written, new row
+    del kv, k, k1
+    torch.cuda.empty_cache()
+    return {"metric": "copy-on-write append GB/s", "value": world * moved / (t * 1e-3) / 1e9, "unit": "GB/s",
+            "ms_per_call": t, "bytes_per_call": moved, "pages_copied": B * w.hkv,
+            "step": "append 1 token to 64 forks of 1000-token sequences (8 heads each: 512 shared pages copied)",
+            "roofline": {"bound": "hbm", "achieved": moved / (t * 1e-3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": moved / (t * 1e-3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                         "kernel": "cow_copy_kernel + append_kernel (events around segkv_append)"}}
 
 
 def bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk):

@@ -13,6 +13,8 @@
 #include <cstring>
 #include <new>
 #include <string>
+#include <unordered_map>
+#include <utility>
 #include <vector>
 
 #include "../../include/segkv.h"
@@ -72,6 +74,12 @@ struct segkv {
   segkv_config cfg;
   std::vector<uint8_t> cls;  // [layers * hkv]
   std::vector<int32_t> len;  // [layers * max_seqs]
+  // Host mirror of the page table in free-list-index space: which free-list entry each
+  // (layer, seq, head, slot) holds (-1: none), and how many slots hold each entry.  It lets
+  // the host plan every allocation, including the copies on write after a fork.
+  std::vector<int32_t> slot_k;  // [layers * max_seqs * hkv * max_lp]
+  std::vector<int32_t> ref;     // [num_pages]
+  long long n_shared = 0;       // entries with ref >= 2: while 0, no append copies a page
   int ring = 0, max_lp = 0, G = 0;
   long long pages_used = 0;
   Staging slot[kStagingSlots];
@@ -111,12 +119,6 @@ StorageGeom geom(const segkv_t *h) {
   g.ring = h->ring;
   g.window = h->cfg.window;
   return g;
-}
-
-// Pages a head holds once its sequence has `n` tokens.
-int held_pages(const segkv_t *h, bool global, int n) {
-  const int full = ceil_div(n, h->cfg.page_size);
-  return global ? full : std::min(full, h->ring);
 }
 
 // Pinned staging slot big enough for `bytes`; waits for the copy that last used it.
@@ -361,6 +363,8 @@ int segkv_create(const segkv_config *c, segkv_t **out) {
   h->cls.assign(c->head_class, c->head_class + (size_t)c->num_layers * c->num_kv_heads);
   for (uint8_t &x : h->cls) x = x ? 1 : 0;
   h->len.assign((size_t)c->num_layers * c->max_seqs, 0);
+  h->slot_k.assign((size_t)c->num_layers * c->max_seqs * c->num_kv_heads * h->max_lp, -1);
+  h->ref.assign((size_t)c->num_pages, 0);
   h->cfg.head_class = nullptr;
   *out = h;
   return SEGKV_OK;
@@ -390,7 +394,10 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
   if (!h || max_batch < 1 || max_tokens < 0) return 0;
   const size_t H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
   const int tile_pos = kPrefillItemRows / h->G;
-  const size_t app = kHeaderBytes + sizeof(AppendSeq) * max_batch + align_up(H, 4) + 4 * H * max_batch;
+  // append: per (sequence, head) the plan offset, then one plan entry per touched page
+  const size_t app = align_up(kHeaderBytes + sizeof(AppendSeq) * max_batch + align_up(H, 4) + 4 * (H * max_batch + 1),
+                              16) +
+                     sizeof(int4) * H * ((size_t)ceil_div(max_tokens, h->cfg.page_size) + 2 * max_batch);
   const size_t pre = prefill_meta_bytes(max_batch, H * ((size_t)ceil_div(max_tokens, tile_pos) + max_batch) +
                                                       kMaxPartSlots, kMaxPartSlots) +
                      prefill_part_bytes((int)D);
@@ -406,7 +413,36 @@ int segkv_reset(segkv_t *h, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   SEGKV_CUDA(h, "reset launch", launch_reset(geom(h), h->cfg.num_layers, static_cast<cudaStream_t>(stream)));
   std::fill(h->len.begin(), h->len.end(), 0);
+  std::fill(h->slot_k.begin(), h->slot_k.end(), -1);
+  std::fill(h->ref.begin(), h->ref.end(), 0);
+  h->n_shared = 0;
   h->pages_used = 0;
+  return SEGKV_OK;
+}
+
+int segkv_fork(segkv_t *h, int src_seq, int dst_seq, void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  const segkv_config &c = h->cfg;
+  if (src_seq < 0 || dst_seq < 0 || src_seq >= c.max_seqs || dst_seq >= c.max_seqs || src_seq == dst_seq)
+    return SEGKV_ERR_INVALID_ARG;
+  for (int l = 0; l < c.num_layers; ++l)
+    if (h->len[(size_t)l * c.max_seqs + dst_seq] != 0) return SEGKV_ERR_INVALID_ARG;
+  const size_t row = (size_t)c.num_kv_heads * h->max_lp;  // one (layer, seq) block of the page table
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int l = 0; l < c.num_layers; ++l)
+    SEGKV_CUDA(h, "fork page-table copy",
+               cudaMemcpyAsync(c.page_table + ((size_t)l * c.max_seqs + dst_seq) * row,
+                               c.page_table + ((size_t)l * c.max_seqs + src_seq) * row, row * sizeof(int32_t),
+                               cudaMemcpyDeviceToDevice, st));
+  for (int l = 0; l < c.num_layers; ++l) {
+    const int32_t *a = &h->slot_k[((size_t)l * c.max_seqs + src_seq) * row];
+    int32_t *b = &h->slot_k[((size_t)l * c.max_seqs + dst_seq) * row];
+    for (size_t i = 0; i < row; ++i) {
+      b[i] = a[i];
+      if (a[i] >= 0 && ++h->ref[a[i]] == 2) h->n_shared++;
+    }
+    h->len[(size_t)l * c.max_seqs + dst_seq] = h->len[(size_t)l * c.max_seqs + src_seq];
+  }
   return SEGKV_OK;
 }
 
@@ -418,26 +454,81 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
   if (rc) return rc;
   if (!start_pos || !num_new) return SEGKV_ERR_INVALID_ARG;
   const int H = h->cfg.num_kv_heads;
-  long long total = 0, new_pages = 0;
-  std::vector<int32_t> pair_off((size_t)nseq * H);  // pages allocated for earlier (sequence, head) pairs
+  long long total = 0;
   for (int b = 0; b < nseq; ++b) {
     const int s = seq_ids[b];
     const int cur = h->len[(size_t)layer * h->cfg.max_seqs + s];
     if (num_new[b] < 0 || start_pos[b] != cur || (long long)cur + num_new[b] > h->cfg.max_seq_len)
       return SEGKV_ERR_INVALID_ARG;
     total += num_new[b];
-    for (int k = 0; k < H; ++k) {
-      const bool global = h->cls[layer * H + k] != 0;
-      pair_off[(size_t)b * H + k] = (int32_t)new_pages;
-      new_pages += held_pages(h, global, cur + num_new[b]) - held_pages(h, global, cur);
-    }
   }
   if (total > (1LL << 30)) return SEGKV_ERR_UNSUPPORTED;
   if (total > 0 && (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16))) return SEGKV_ERR_INVALID_ARG;
+  // Page plan, in the allocation order (sequence in call order, head ascending, logical page
+  // ascending): for every page the call touches, the free-list index of a page it takes --
+  // the slot is empty, or its page is shared with another sequence (copy on write: the
+  // rows before the call's first token on that page are copied over) -- or -1 (the slot's
+  // page is this sequence's alone and is written in place).
+  const int P = h->cfg.page_size, R = h->ring, max_lp = h->max_lp;
+  // Logical pages [lp0, lp1] the call touches for (sequence b, head k), and the mirror row.
+  auto touched = [&](int b, int k, int &lp0, int &lp1, size_t &row, bool &global) {
+    global = h->cls[layer * H + k] != 0;
+    lp1 = (start_pos[b] + num_new[b] - 1) / P;
+    lp0 = start_pos[b] / P;
+    if (!global && lp1 - R + 1 > lp0) lp0 = lp1 - R + 1;
+    row = (((size_t)layer * h->cfg.max_seqs + seq_ids[b]) * H + k) * max_lp;
+  };
+  std::vector<int32_t> pair_page((size_t)nseq * H + 1, 0);  // first plan entry of each pair
+  std::vector<int32_t> pair_new((size_t)nseq * H + 1, 0);   // pages allocated for earlier pairs
+  std::vector<int32_t> plan;
+  std::vector<int4> jobs;  // (k_new, k_old, rows before the call's first token)
+  const bool copies = h->n_shared > 0;  // else every page is one sequence's: no copy, no plan
+  // changes to the mirror, applied once the call is accepted; refcounts seen through them, so
+  // a page one sequence of the call copies is no longer shared for a later one
+  std::vector<std::pair<size_t, int32_t>> slot_set;
+  std::unordered_map<int32_t, int32_t> ref_delta;
+  auto ref_of = [&](int32_t k) {
+    const auto it = ref_delta.find(k);
+    return h->ref[k] + (it == ref_delta.end() ? 0 : it->second);
+  };
+  long long new_pages = 0;
+  for (int b = 0; b < nseq; ++b)
+    for (int k = 0; k < H; ++k) {
+      pair_page[(size_t)b * H + k] = (int32_t)plan.size();
+      pair_new[(size_t)b * H + k] = (int32_t)new_pages;
+      if (num_new[b] == 0) continue;
+      int lp0, lp1;
+      size_t row;
+      bool global;
+      touched(b, k, lp0, lp1, row, global);
+      if (!copies) {  // a page is taken exactly for an empty slot
+        for (int lp = lp0; lp <= lp1; ++lp) new_pages += h->slot_k[row + (global ? lp : lp % R)] < 0;
+        continue;
+      }
+      const int first = start_pos[b];
+      for (int lp = lp0; lp <= lp1; ++lp) {
+        const size_t idx = row + (global ? lp : lp % R);
+        const int32_t k_old = h->slot_k[idx];
+        if (k_old >= 0 && ref_of(k_old) <= 1) {
+          plan.push_back(-1);
+          continue;
+        }
+        const int32_t k_new = (int32_t)(h->pages_used + new_pages++);
+        const int copy_rows = (k_old >= 0 && lp == first / P) ? first % P : 0;
+        plan.push_back(k_new);
+        if (copy_rows > 0) jobs.push_back(make_int4(k_new, k_old, copy_rows, 0));
+        slot_set.push_back({idx, k_new});
+        if (k_old >= 0) ref_delta[k_old] -= 1;
+      }
+    }
+  pair_page[(size_t)nseq * H] = (int32_t)plan.size();
+  pair_new[(size_t)nseq * H] = (int32_t)new_pages;
   if (h->pages_used + new_pages > h->cfg.num_pages) return SEGKV_ERR_OUT_OF_PAGES;
   const size_t cls_off = kHeaderBytes + sizeof(AppendSeq) * nseq;
   const size_t off_off = cls_off + align_up(H, 4);
-  const size_t bytes = off_off + 4 * (size_t)H * nseq;
+  const size_t plan_off = align_up(off_off + 4 * ((size_t)H * nseq + 1), 16);
+  const size_t jobs_off = align_up(plan_off + 4 * plan.size(), 16);
+  const size_t bytes = jobs_off + sizeof(int4) * jobs.size();
   if (!ws || !aligned(ws, 256) || ws_bytes < bytes) return SEGKV_ERR_WORKSPACE;
   if ((rc = ensure_device_state(h))) return rc;
   if (total == 0) return SEGKV_OK;
@@ -451,14 +542,45 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
     tok += num_new[b];
   }
   std::memcpy(static_cast<char *>(host) + cls_off, &h->cls[(size_t)layer * H], H);
-  std::memcpy(static_cast<char *>(host) + off_off, pair_off.data(), 4 * (size_t)H * nseq);
+  std::memcpy(static_cast<char *>(host) + off_off, copies ? pair_page.data() : pair_new.data(), 4 * pair_page.size());
+  if (!plan.empty()) std::memcpy(static_cast<char *>(host) + plan_off, plan.data(), 4 * plan.size());
+  if (!jobs.empty()) std::memcpy(static_cast<char *>(host) + jobs_off, jobs.data(), sizeof(int4) * jobs.size());
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = upload(h, ws, bytes, st))) return rc;
   const uint8_t *cls_dev = static_cast<const uint8_t *>(ws) + cls_off;
   const int32_t *off_dev = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + off_off);
+  const int32_t *plan_dev = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + plan_off);
+  const int4 *jobs_dev = reinterpret_cast<const int4 *>(static_cast<const char *>(ws) + jobs_off);
   SEGKV_CUDA(h, "append launch",
-             launch_append(geom(h), layer, ws, nseq, cls_dev, off_dev, (int)h->pages_used, (int)new_pages, (int)total,
-                           k_new, v_new, st));
+             launch_append(geom(h), layer, ws, nseq, cls_dev, off_dev, copies ? plan_dev : nullptr, jobs_dev,
+                           (int)jobs.size(), (int)h->pages_used, (int)new_pages, (int)total, k_new, v_new, st));
+  if (copies) {
+    for (const auto &e : slot_set) {
+      h->slot_k[e.first] = e.second;
+      h->ref[e.second] = 1;
+    }
+    for (const auto &e : ref_delta) {
+      const int32_t before = h->ref[e.first];
+      h->ref[e.first] += e.second;
+      if (before >= 2 && h->ref[e.first] < 2) h->n_shared--;
+    }
+  } else {  // the kernel's closed form: new pages in the allocation order
+    int32_t k_new = (int32_t)h->pages_used;
+    for (int b = 0; b < nseq; ++b)
+      for (int k = 0; k < H && num_new[b] > 0; ++k) {
+        int lp0, lp1;
+        size_t row;
+        bool global;
+        touched(b, k, lp0, lp1, row, global);
+        for (int lp = lp0; lp <= lp1; ++lp) {
+          int32_t &slot = h->slot_k[row + (global ? lp : lp % R)];
+          if (slot < 0) {
+            slot = k_new;
+            h->ref[k_new++] = 1;
+          }
+        }
+      }
+  }
   for (int b = 0; b < nseq; ++b) h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] += num_new[b];
   h->pages_used += new_pages;
   return SEGKV_OK;

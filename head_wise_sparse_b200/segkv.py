@@ -25,7 +25,7 @@ EXPORTS = [
     "segkv_create", "segkv_destroy", "segkv_ring_pages", "segkv_max_lp", "segkv_seq_len", "segkv_pages_used",
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
     "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
-    "segkv_decode_attn_noalloc", "segkv_relocate_q",
+    "segkv_decode_attn_noalloc", "segkv_relocate_q", "segkv_fork",
 ]
 
 
@@ -74,6 +74,7 @@ def lib():
         L.segkv_decode_attn.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P, SZ, P]
         L.segkv_decode_attn_noalloc.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P]
         L.segkv_relocate_q.argtypes = [P, I, I, P, P, P, F, I, P]
+        L.segkv_fork.argtypes = [P, I, I, P]
         L.segkv_device_status.argtypes = [P, P]
         L.segkv_last_error.argtypes = [P]
         L.segkv_last_error.restype = ctypes.c_char_p
@@ -183,6 +184,9 @@ class Handle:
                                                int(num_splits), _dptr(out), _dptr(lse), _dptr(visited),
                                                _stream(stream))
 
+    def fork(self, src_seq, dst_seq, stream=None) -> None:
+        _check(lib().segkv_fork(self.h, int(src_seq), int(dst_seq), _stream(stream)), "segkv_fork", self.h)
+
     def relocate_q(self, layer, n_tokens, shift, q_in, q_out, theta_base, interleaved, stream=None) -> int:
         return lib().segkv_relocate_q(self.h, layer, int(n_tokens), _dptr(shift), _dptr(q_in), _dptr(q_out),
                                       float(theta_base), int(interleaved), _stream(stream))
@@ -268,6 +272,10 @@ class SegKV:
         _check(self.handle.decode(layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, self.ws,
                                   self.ws_bytes), "segkv_decode_attn", self.handle.h)
         return out, lse
+
+    def fork(self, src_seq: int, dst_seq: int) -> None:
+        """segkv_fork: dst_seq (empty) shares src_seq's pages; appends copy shared pages first."""
+        self.handle.fork(src_seq, dst_seq)
 
     def relocate_q(self, layer: int, q, shift, *, out=None, theta_base: float = 10000.0, interleaved: bool = False):
         """segkv_relocate_q: local heads' queries turned by the rotary angle of position -shift

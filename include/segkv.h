@@ -107,14 +107,27 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens);
 int segkv_reset(segkv_t *h, void *stream);
 
 /*
+ * Fork (hysenlabs.com write-up, "Experimental Features and Current Limitations": a shared KV
+ * manager with forks and copy-on-write append): the empty sequence dst_seq takes src_seq's
+ * page-table rows and length in every layer, so the two share those pages (reference
+ * counted in the handle).  A later append to either one that touches a shared page first
+ * gives that sequence a private copy (see segkv_append), so neither sees the other's new
+ * tokens.  Enqueues one device-to-device copy of the page-table rows per layer.
+ * Errors: INVALID_ARG (ids out of range, src == dst, dst not empty in some layer), CUDA.
+ */
+int segkv_fork(segkv_t *h, int src_seq, int dst_seq, void *stream);
+
+/*
  * Appends tokens [start_pos[b], start_pos[b] + num_new[b]) of sequence seq_ids[b] to every
  * KV head of `layer`: the per-head page tables grow and the K/V rows are scattered into the
  * pages (zhichai.net news item "What Happened", item 3: per-(layer, head) segmented paged
  * storage).  start_pos[b] must equal segkv_seq_len(h, layer, seq_ids[b]); seq ids
  * in one call are distinct.  k_new / v_new: DEVICE bf16 [sum(num_new), Hkv, D],
  * sequences packed in call order.
- *   Page rule: every unallocated slot touched takes the next id of the free list, in the
- *   order (sequence in call order, KV head ascending, logical page ascending).  A global
+ *   Page rule: every slot touched that is unallocated, or whose page another sequence
+ *   shares after a fork, takes the next id of the free list, in the order (sequence in call
+ *   order, KV head ascending, logical page ascending); a shared page's rows before the
+ *   call's first token are copied into the new page (copy on write).  A global
  *   head stores logical page lp in slot lp; a local head in slot lp mod R and keeps only
  *   the last R logical pages ending at the call's last token (older tokens of the call
  *   are skipped: the ring would overwrite them).  The unwritten rows of a page the call

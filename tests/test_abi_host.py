@@ -76,6 +76,15 @@ def test_append_validation_happens_before_any_enqueue():
     assert h.seq_len(0, 0) == 0 and h.pages_used == 0
 
 
+def test_fork_validation_happens_before_any_enqueue():
+    h = handle()
+    for src, dst in ((0, 0), (-1, 1), (0, 4), (4, 0)):
+        with pytest.raises(segkv.SegkvError) as e:
+            h.fork(src, dst, stream=0)
+        assert e.value.code == 1
+    assert h.seq_len(0, 1) == 0
+
+
 def test_attention_validation_happens_before_any_enqueue():
     h = handle()
     big = 1 << 20

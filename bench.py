@@ -475,7 +475,10 @@ def bench_fork(args, torch, dev, stream, max_over_ranks, world, pk):
 
 
 def bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk):
-    """Batched decode: 64 sequences, context 32767 (+1 new token per step), split-K + combine."""
+    """Batched decode: 64 sequences, context 32767 (+1 new token per step).  The step runs
+    first as the fused segkv_decode_step (the split kernel appends the token itself; split +
+    combine), which gives the line's value, then as two calls (segkv_append of the token,
+    then segkv_decode_attn: append kernel, split kernel, combine kernel) for comparison."""
     from head_wise_sparse_b200.segkv import SegKV
 
     w = wl.CONFIGS[DECODE]
@@ -483,8 +486,9 @@ def bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk):
     ctx = w.seqs[0].context
     steps = min(args.steps, 100)
     warm = args.warmup
-    max_len = ctx + steps + warm + 64
-    wmax = w.scaled(seqs=tuple(wl.Seq(ctx, steps + warm + 1, ctx, ctx + 1) for _ in range(B)))
+    nsteps = warm + steps
+    max_len = ctx + 2 * nsteps + 64
+    wmax = w.scaled(seqs=tuple(wl.Seq(ctx, 2 * nsteps + 1, ctx, ctx + 1) for _ in range(B)))
     kv = SegKV(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=w.page, window=w.window,
                head_class=w.class_array(), num_pages=wmax.num_pages, free_list=wmax.free_list(), max_seqs=B,
                max_seq_len=max_len, ring_pages=w.ring_pages, max_chunk=1, ws_batch=B, ws_tokens=B * 2048, device=dev)
@@ -498,10 +502,9 @@ def bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk):
         v = torch.randn((B * n, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
         kv.append(0, ids, [lo] * B, [n] * B, k, v)
         del k, v
-    nsteps = warm + steps
-    k_new = torch.randn((nsteps, B, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
-    v_new = torch.randn((nsteps, B, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
-    q = torch.randn((nsteps, B, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    k_new = torch.randn((2 * nsteps, B, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    v_new = torch.randn((2 * nsteps, B, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn((2 * nsteps, B, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
     out = torch.empty((B, w.hq, w.d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, w.hq), dtype=torch.float32, device=dev)
     n_glob = int(sum(w.classes[0]))
@@ -510,39 +513,53 @@ def bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk):
         keys = n_glob * (p + 1) + (w.hkv - n_glob) * min(p + 1, w.window)
         return B * keys * w.d * 2 * 2
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    total_bytes = 0
-    for s in range(nsteps):
-        p = ctx + s
-        timed = s >= warm
-        if timed and s == warm:
-            barrier()
-            torch.cuda.synchronize()
-        if timed:
-            ev[s - warm][0].record(stream)
-        kv.append(0, ids, [p] * B, [1] * B, k_new[s], v_new[s])
-        if timed:
-            ev[s - warm][1].record(stream)
-        kv.decode(0, ids, [p] * B, q[s], out=out, lse=lse)
-        if timed:
-            ev[s - warm][2].record(stream)
-            total_bytes += kv_bytes(p)
-    torch.cuda.synchronize()
-    barrier()
+    def run(fused, s0):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        total_bytes = 0
+        for i in range(nsteps):
+            s = s0 + i
+            p = ctx + s
+            timed = i >= warm
+            if timed and i == warm:
+                barrier()
+                torch.cuda.synchronize()
+            if timed:
+                ev[i - warm][0].record(stream)
+            if fused:
+                kv.decode_step(0, ids, k_new[s], v_new[s], q[s], out=out, lse=lse)
+                if timed:
+                    ev[i - warm][1].record(stream)
+            else:
+                kv.append(0, ids, [p] * B, [1] * B, k_new[s], v_new[s])
+                if timed:
+                    ev[i - warm][1].record(stream)
+                kv.decode(0, ids, [p] * B, q[s], out=out, lse=lse)
+            if timed:
+                ev[i - warm][2].record(stream)
+                total_bytes += kv_bytes(p)
+        torch.cuda.synchronize()
+        barrier()
+        t_step = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in ev) / steps)
+        t_dec = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / steps)
+        return t_step, t_dec, total_bytes / steps
+
+    t_step, _, per_step = run(True, 0)  # the fused step first, at the configured context
+    t_pair, t_pair_dec, b_pair = run(False, nsteps)
     if kv.device_status() != 0:
         raise RuntimeError("device error word set during decode")
-    t_step = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in ev) / steps)
-    t_dec = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / steps)
-    per_step = total_bytes / steps
-    achieved = per_step / (t_dec * 1e-3) / 1e9
+    achieved = per_step / (t_step * 1e-3) / 1e9
     res = {
         "workload": DECODE, "metric": "decode KV GB/s", "value": world * per_step / (t_step * 1e-3) / 1e9,
-        "unit": "GB/s", "ms_per_step": t_step, "decode_kernel_ms": t_dec, "steps": steps,
-        "kv_bytes_per_step": per_step, "step": "append 1 token/seq (page ids + scatter) + split-K decode + combine",
+        "unit": "GB/s", "ms_per_step": t_step, "steps": steps, "kv_bytes_per_step": per_step,
+        "step": "segkv_decode_step: the split kernel appends each sequence's token, then split-K decode + combine",
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic("decode_64x32k.md", DECODE_SOURCES),
-                     "kernel": "decode_split_kernel<128> + lse_combine (events around segkv_decode_attn)"},
-        "gpu_launches": 3 * steps, "data": "synthetic (seeded torch generator on the device)",
+                     "kernel": "decode_split_kernel<128> with the step's append + lse_combine "
+                               "(events around segkv_decode_step)"},
+        "two_calls": {"value": world * b_pair / (t_pair * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": t_pair,
+                      "decode_ms": t_pair_dec, "step": "segkv_append (1 token) + segkv_decode_attn",
+                      "gpu_launches": 3 * steps},
+        "gpu_launches": 2 * steps, "data": "synthetic (seeded torch generator on the device)",
     }
     del kv
     torch.cuda.empty_cache()

@@ -12,7 +12,14 @@
 // into a 6-deep ring; warps 0..3 each take 16 keys of every stage, keep their own running
 // max / sum / output, and merge at the end of the item.  The merged partial (output
 // normalised by its own sum, and its natural-log lse) goes to the workspace; the combine
-// kernel folds the splits of each (sequence, query head).
+// kernel folds the splits of each (sequence, query head).  It is chained to the split
+// kernel by programmatic dependent launch, so its CTAs are resident and waiting when the
+// split kernel ends.
+//
+// Decode step: the same kernel also appends the step's token.  Only the item holding a
+// head's last page reads the row at q_pos, so that item's producer warp writes the K and V
+// rows (and, for a page the token starts, the page-table entry and the zeroed rest of the
+// page) before it loads the page; a proxy fence orders those stores before the TMA reads.
 #include "device_common.cuh"
 
 namespace skv {
@@ -67,6 +74,43 @@ __device__ __forceinline__ DItem decode_ditem(const DecodeLaunch &p, const Decod
   const int pps = kKeys / P;
   it.n_stages = (it.lp_b - it.lp_a + 1 + pps - 1) / pps;
   return it;
+}
+
+// Decode step, producer warp of the item that holds the last page of (sequence, KV head):
+// writes the token's K and V rows at q_pos and returns the page's id (num_pages after a
+// bad page id, which sets the error word; the TMA then reads zeros).
+template <int D>
+__device__ int step_append(const DecodeLaunch &p, const DItem &it, long long row_base, int lane, int32_t *state) {
+  constexpr int CH = D / 8;
+  const int P = p.g.page, pos = it.q_pos, lp = pos / P;
+  const long long slot = row_base + (it.global ? lp : lp % p.g.ring);
+  const int k = p.newk[it.b * p.g.hkv + it.h];
+  int32_t phys;
+  if (k >= 0) phys = k < p.g.num_pages ? p.g.free_list[k] : -1;
+  else phys = p.g.page_table[slot];
+  if (phys < 0 || phys >= p.g.num_pages) {
+    if (lane == 0) set_error(state, kErrDeviceBounds);
+    return p.g.num_pages;
+  }
+  if (k >= 0 && lane == 0) p.g.page_table[slot] = phys;
+  uint4 *kp = reinterpret_cast<uint4 *>(p.g.k_pool);
+  uint4 *vp = reinterpret_cast<uint4 *>(p.g.v_pool);
+  const long long src = ((long long)it.b * p.g.hkv + it.h) * CH;
+  const long long row = (long long)phys * P + pos % P;
+  for (int e = lane; e < 2 * CH; e += 32) {
+    if (e < CH) kp[row * CH + e] = static_cast<const uint4 *>(p.k_new)[src + e];
+    else vp[row * CH + e - CH] = static_cast<const uint4 *>(p.v_new)[src + e - CH];
+  }
+  if (pos % P == 0) {  // a page the token starts: the rows after it hold zeros
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int e = lane; e < (P - 1) * CH; e += 32) {
+      kp[(row + 1) * CH + e] = z;
+      vp[(row + 1) * CH + e] = z;
+    }
+  }
+  fence_async_global();
+  __syncwarp();
+  return phys;
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
@@ -126,6 +170,8 @@ __global__ void __launch_bounds__(kThreadsDec, 1)
     mbar_init(&bar->merge[1], 128);
     bar->abort_flag = 0;
     fence_mbar_init();
+    if (p.newk && blockIdx.x == 0) state[0] = p.cursor_after;
+    pdl_launch_dependents();  // the combine kernel may start its CTAs; they wait for this grid
   }
   __syncthreads();
 
@@ -153,6 +199,8 @@ __global__ void __launch_bounds__(kThreadsDec, 1)
       const DItem it = decode_ditem(p, seqs, items, idx);
       const long long row_base = (((long long)p.layer * p.g.max_seqs + it.seq_id) * p.g.hkv + it.h) * p.g.max_lp;
       const int last_lp = it.hi / P;  // every key of the query is stored (host-validated)
+      // decode step: the item holding the last page writes the token's row first
+      const int last_phys = (p.newk && it.lp_b == last_lp) ? step_append<D>(p, it, row_base, lane, state) : -1;
       int lp_base = -(1 << 30), pid = p.g.num_pages;
       for (int j = 0; j < it.n_stages; ++j) {
         const int lp_first = it.lp_a + j * pps;
@@ -160,13 +208,14 @@ __global__ void __launch_bounds__(kThreadsDec, 1)
           lp_base = lp_first;
           const int lp = lp_base + lane;
           pid = p.g.num_pages;
-          if (lp <= it.lp_b) {
+          if (last_phys >= 0 && lp == last_lp) {
+            pid = last_phys;
+          } else if (lp <= it.lp_b) {
             const int32_t v = p.g.page_table[row_base + (it.global ? lp : lp % p.g.ring)];
             if (v >= 0 && v < p.g.num_pages) pid = v;
             else set_error(state, kErrDeviceBounds);
           }
         }
-        (void)last_lp;
         const int s = c % kStagesDec;
         const uint32_t u = (uint32_t)(c / kStagesDec);
         if (!(ok = warp_wait(&bar->empty[s], (u & 1) ^ 1, abort_flag, state))) break;
@@ -354,6 +403,7 @@ __global__ void __launch_bounds__(kThreadsDec, 1)
 // out = sum exp(lse_i - lse) * out_i, rounded once to bf16.
 template <int D>
 __global__ void __launch_bounds__(128) lse_combine_kernel(const DecodeLaunch p, const int32_t *__restrict__ nsplit) {
+  pdl_wait_primary();  // the split kernel's partials are complete and visible
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= p.nseq * p.g.hq) return;
@@ -390,33 +440,38 @@ __global__ void __launch_bounds__(128) lse_combine_kernel(const DecodeLaunch p, 
 
 int decode_smem_bytes(int head_dim) { return head_dim == 64 ? DSmem<64>::kBytes : DSmem<128>::kBytes; }
 
-cudaError_t launch_decode(const DecodeLaunch &p, const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t st) {
-  static bool attr_set[2] = {false, false};
-  const int smem = decode_smem_bytes(p.g.head_dim);
+template <int D>
+cudaError_t launch_decode_d(const DecodeLaunch &p, const CUtensorMap &kmap, const CUtensorMap &vmap, int smem,
+                            cudaStream_t st) {
+  static bool attr_set = false;
+  cudaError_t e;
+  if (!attr_set) {
+    if ((e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+      return e;
+    attr_set = true;
+  }
+  decode_split_kernel<D><<<p.grid, kThreadsDec, smem, st>>>(kmap, vmap, p);
+  if ((e = cudaGetLastError())) return e;
   const int32_t *nsplit =
       reinterpret_cast<const int32_t *>(static_cast<const char *>(p.ws_meta) + p.nsplit_off);
   const int rows = p.nseq * p.g.hq;
-  cudaError_t e;
-  if (p.g.head_dim == 64) {
-    if (!attr_set[0]) {
-      if ((e = cudaFuncSetAttribute(decode_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
-        return e;
-      attr_set[0] = true;
-    }
-    decode_split_kernel<64><<<p.grid, kThreadsDec, smem, st>>>(kmap, vmap, p);
-    if ((e = cudaGetLastError())) return e;
-    lse_combine_kernel<64><<<(rows + 3) / 4, 128, 0, st>>>(p, nsplit);
-  } else {
-    if (!attr_set[1]) {
-      if ((e = cudaFuncSetAttribute(decode_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
-        return e;
-      attr_set[1] = true;
-    }
-    decode_split_kernel<128><<<p.grid, kThreadsDec, smem, st>>>(kmap, vmap, p);
-    if ((e = cudaGetLastError())) return e;
-    lse_combine_kernel<128><<<(rows + 3) / 4, 128, 0, st>>>(p, nsplit);
-  }
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((rows + 3) / 4);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, lse_combine_kernel<D>, p, nsplit);
+}
+
+cudaError_t launch_decode(const DecodeLaunch &p, const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t st) {
+  const int smem = decode_smem_bytes(p.g.head_dim);
+  return p.g.head_dim == 64 ? launch_decode_d<64>(p, kmap, vmap, smem, st)
+                            : launch_decode_d<128>(p, kmap, vmap, smem, st);
 }
 
 }  // namespace skv

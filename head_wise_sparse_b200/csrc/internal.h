@@ -93,6 +93,13 @@ struct DecodeLaunch {
   float *lse;
   unsigned long long *visited;
   float scale_log2;
+  // Decode step (newk != NULL): before attending, each (sequence, KV head) appends its token
+  // at q_pos: newk[b * hkv + h] = free-list entry of a page the token starts (-1: the slot's
+  // page is written in place); K/V rows from k_new / v_new [nseq, hkv, D]; block 0 sets the
+  // allocation cursor state[0] = cursor_after.
+  const int32_t *newk;
+  const void *k_new, *v_new;
+  int cursor_after;
 };
 cudaError_t launch_decode(const DecodeLaunch &p, const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t st);
 int decode_smem_bytes(int head_dim);

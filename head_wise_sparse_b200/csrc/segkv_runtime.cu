@@ -315,6 +315,111 @@ size_t prefill_part_bytes(int head_dim) {
   return (size_t)kMaxPartSlots * 2 * 128 * ((size_t)head_dim + 1) * 4;
 }
 
+// The token of a decode step, appended by the decode kernel itself: newk[b * hkv + h] =
+// free-list entry of a page the token starts (-1: written in place), K/V rows on the device.
+struct StepRows {
+  const std::vector<int32_t> *newk;
+  const void *k_new, *v_new;
+  int cursor_after;
+};
+
+// Decode planning and launch.  With `step`, every sequence's length counts the step's token
+// (not yet in the host's lengths) and the kernel appends it before attending.
+int decode_common(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos, const void *q,
+                  float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited, void *ws,
+                  size_t ws_bytes, void *stream, const StepRows *step) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  int rc = check_seqs(h, layer, nseq, seq_ids);
+  if (rc) return rc;
+  if (!q_pos || num_splits < 0) return SEGKV_ERR_INVALID_ARG;
+  if (h->G > 16) return SEGKV_ERR_UNSUPPORTED;
+  if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4)) return SEGKV_ERR_INVALID_ARG;
+  const int P = h->cfg.page_size, H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
+  const bool has_local = layer_has_local(h, layer);
+  long long total_pages = 0;
+  int max_pages = 0;
+  for (int b = 0; b < nseq; ++b) {
+    const int len = h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] + (step ? 1 : 0);
+    if (q_pos[b] < 0 || q_pos[b] >= len) return SEGKV_ERR_INVALID_ARG;
+    if (has_local && !ring_covers(h, len, q_pos[b])) return SEGKV_ERR_RING_TOO_SMALL;
+    for (int k = 0; k < H; ++k) {
+      const int lo = h->cls[layer * H + k] ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
+      const int n = q_pos[b] / P - lo / P + 1;
+      total_pages += n;
+      max_pages = std::max(max_pages, n);
+    }
+  }
+  if ((rc = ensure_device_state(h))) return rc;
+  // split size in pages: a multiple of the pages of one 64-key stage
+  const int pps = kDecodeStageKeys / P;
+  int split;
+  if (num_splits > 0) {
+    split = ceil_div(max_pages, std::min(num_splits, kMaxSplits));
+  } else {
+    const long long target = std::max<long long>(1, total_pages / (8LL * h->num_sms));
+    split = 1;
+    while (2LL * split <= target && split < 256) split *= 2;
+  }
+  split = std::max(split, ceil_div(max_pages, kMaxSplits));
+  split = ceil_div(split, pps) * pps;
+  const int max_splits = ceil_div(max_pages, split);
+  const int nsplit_off = kHeaderBytes + (int)sizeof(DecodeSeq) * nseq;
+  const int newk_off = nsplit_off + 4 * nseq * H;
+  const int items_off = (int)align_up(newk_off + (step ? 4 * nseq * H : 0), 16);
+  std::vector<int2> items;
+  std::vector<int32_t> nsplit((size_t)nseq * H);
+  for (int b = 0; b < nseq; ++b)
+    for (int k = 0; k < H; ++k) {
+      const bool global = h->cls[layer * H + k] != 0;
+      const int lo = global ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
+      const int n = ceil_div(q_pos[b] / P - lo / P + 1, split);
+      nsplit[(size_t)b * H + k] = n;
+      for (int s = 0; s < n; ++s) items.push_back(make_int2(b, (int)make_item_w1(global, k, s)));
+    }
+  const size_t meta_bytes = items_off + 8 * items.size();
+  const size_t part_o_off = align_up(meta_bytes, 256);
+  const size_t part_lse_off = part_o_off + align_up(4 * (size_t)nseq * Hq * max_splits * D, 256);
+  const size_t need = part_lse_off + 4 * (size_t)nseq * Hq * max_splits;
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEGKV_ERR_WORKSPACE;
+  void *host = nullptr;
+  if ((rc = staging(h, meta_bytes, &host))) return rc;
+  std::memset(host, 0, items_off);
+  DecodeSeq *ds = reinterpret_cast<DecodeSeq *>(static_cast<char *>(host) + kHeaderBytes);
+  for (int b = 0; b < nseq; ++b)
+    ds[b] = DecodeSeq{seq_ids[b], q_pos[b], h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] + (step ? 1 : 0), 0};
+  std::memcpy(static_cast<char *>(host) + nsplit_off, nsplit.data(), 4 * nsplit.size());
+  if (step) std::memcpy(static_cast<char *>(host) + newk_off, step->newk->data(), 4 * step->newk->size());
+  std::memcpy(static_cast<char *>(host) + items_off, items.data(), 8 * items.size());
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = upload(h, ws, meta_bytes, st))) return rc;
+  DecodeLaunch p{};  // zeroed: fields a path does not set (the step append) stay off
+  p.g = geom(h);
+  p.layer = layer;
+  p.nseq = nseq;
+  p.n_items = (int)items.size();
+  p.split_pages = split;
+  p.max_splits = max_splits;
+  p.grid = std::min<int>((int)items.size(), h->num_sms);
+  p.ws_meta = ws;
+  p.nsplit_off = nsplit_off;
+  p.items_off = items_off;
+  p.part_o = reinterpret_cast<float *>(static_cast<char *>(ws) + part_o_off);
+  p.part_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + part_lse_off);
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.visited = reinterpret_cast<unsigned long long *>(visited);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.newk = step ? reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + newk_off) : nullptr;
+  p.k_new = step ? step->k_new : nullptr;
+  p.v_new = step ? step->v_new : nullptr;
+  p.cursor_after = step ? step->cursor_after : 0;
+  SEGKV_CUDA(h, "decode launch", launch_decode(p, h->kmap, h->vmap, st));
+  return SEGKV_OK;
+}
+
+
 }  // namespace
 
 // ============================================================================== C ABI
@@ -670,7 +775,7 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
   }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = upload(h, ws, bytes, st))) return rc;
-  PrefillLaunch p;
+  PrefillLaunch p{};
   p.g = geom(h);
   p.layer = layer;
   p.nseq = nseq;
@@ -696,88 +801,63 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
 int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,
                       const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
                       void *ws, size_t ws_bytes, void *stream) {
+  return decode_common(h, layer, nseq, seq_ids, q_pos, q, softmax_scale, num_splits, out, lse, visited, ws, ws_bytes,
+                       stream, nullptr);
+}
+
+int segkv_decode_step(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const void *k_new, const void *v_new,
+                      const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
+                      void *ws, size_t ws_bytes, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   int rc = check_seqs(h, layer, nseq, seq_ids);
   if (rc) return rc;
-  if (!q_pos || num_splits < 0) return SEGKV_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return SEGKV_ERR_INVALID_ARG;
+  if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4) || num_splits < 0)
+    return SEGKV_ERR_INVALID_ARG;
   if (h->G > 16) return SEGKV_ERR_UNSUPPORTED;
-  if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4)) return SEGKV_ERR_INVALID_ARG;
-  const int P = h->cfg.page_size, H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads, D = h->cfg.head_dim;
-  const bool has_local = layer_has_local(h, layer);
-  long long total_pages = 0;
-  int max_pages = 0;
+  const int H = h->cfg.num_kv_heads, P = h->cfg.page_size, R = h->ring;
+  std::vector<int32_t> pos((size_t)nseq);
   for (int b = 0; b < nseq; ++b) {
-    const int len = h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]];
-    if (q_pos[b] < 0 || q_pos[b] >= len) return SEGKV_ERR_INVALID_ARG;
-    if (has_local && !ring_covers(h, len, q_pos[b])) return SEGKV_ERR_RING_TOO_SMALL;
-    for (int k = 0; k < H; ++k) {
-      const int lo = h->cls[layer * H + k] ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
-      const int n = q_pos[b] / P - lo / P + 1;
-      total_pages += n;
-      max_pages = std::max(max_pages, n);
-    }
+    pos[b] = h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]];
+    if (pos[b] + 1 > h->cfg.max_seq_len) return SEGKV_ERR_INVALID_ARG;
+    if (layer_has_local(h, layer) && !ring_covers(h, pos[b] + 1, pos[b])) return SEGKV_ERR_RING_TOO_SMALL;
   }
-  if ((rc = ensure_device_state(h))) return rc;
-  // split size in pages: a multiple of the pages of one 64-key stage
-  const int pps = kDecodeStageKeys / P;
-  int split;
-  if (num_splits > 0) {
-    split = ceil_div(max_pages, std::min(num_splits, kMaxSplits));
-  } else {
-    const long long target = std::max<long long>(1, total_pages / (8LL * h->num_sms));
-    split = 1;
-    while (2LL * split <= target && split < 256) split *= 2;
+  if (h->n_shared > 0) {
+    // a page may be shared after a fork: the append's copy on write runs first, as its own call
+    std::vector<int32_t> one((size_t)nseq, 1);
+    if ((rc = segkv_append(h, layer, nseq, seq_ids, pos.data(), one.data(), k_new, v_new, ws, ws_bytes, stream)))
+      return rc;
+    return segkv_decode_attn(h, layer, nseq, seq_ids, pos.data(), q, softmax_scale, num_splits, out, lse, visited,
+                             ws, ws_bytes, stream);
   }
-  split = std::max(split, ceil_div(max_pages, kMaxSplits));
-  split = ceil_div(split, pps) * pps;
-  const int max_splits = ceil_div(max_pages, split);
-  const int nsplit_off = kHeaderBytes + (int)sizeof(DecodeSeq) * nseq;
-  const int items_off = (int)align_up(nsplit_off + 4 * nseq * H, 16);
-  std::vector<int2> items;
-  std::vector<int32_t> nsplit((size_t)nseq * H);
+  // the append's page rule for one token: a page starts at pos % P == 0 and takes a new
+  // free-list entry unless it recycles a full ring's slot in place
+  std::vector<int32_t> newk((size_t)nseq * H, -1);
+  long long new_pages = 0;
   for (int b = 0; b < nseq; ++b)
     for (int k = 0; k < H; ++k) {
+      const int lp = pos[b] / P;
+      const size_t row = (((size_t)layer * h->cfg.max_seqs + seq_ids[b]) * H + k) * h->max_lp;
       const bool global = h->cls[layer * H + k] != 0;
-      const int lo = global ? 0 : std::max(0, q_pos[b] - h->cfg.window + 1);
-      const int n = ceil_div(q_pos[b] / P - lo / P + 1, split);
-      nsplit[(size_t)b * H + k] = n;
-      for (int s = 0; s < n; ++s) items.push_back(make_int2(b, (int)make_item_w1(global, k, s)));
+      if (h->slot_k[row + (global ? lp : lp % R)] < 0) newk[(size_t)b * H + k] = (int32_t)(h->pages_used + new_pages++);
     }
-  const size_t meta_bytes = items_off + 8 * items.size();
-  const size_t part_o_off = align_up(meta_bytes, 256);
-  const size_t part_lse_off = part_o_off + align_up(4 * (size_t)nseq * Hq * max_splits * D, 256);
-  const size_t need = part_lse_off + 4 * (size_t)nseq * Hq * max_splits;
-  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEGKV_ERR_WORKSPACE;
-  void *host = nullptr;
-  if ((rc = staging(h, meta_bytes, &host))) return rc;
-  std::memset(host, 0, items_off);
-  DecodeSeq *ds = reinterpret_cast<DecodeSeq *>(static_cast<char *>(host) + kHeaderBytes);
-  for (int b = 0; b < nseq; ++b)
-    ds[b] = DecodeSeq{seq_ids[b], q_pos[b], h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]], 0};
-  std::memcpy(static_cast<char *>(host) + nsplit_off, nsplit.data(), 4 * nsplit.size());
-  std::memcpy(static_cast<char *>(host) + items_off, items.data(), 8 * items.size());
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((rc = upload(h, ws, meta_bytes, st))) return rc;
-  DecodeLaunch p;
-  p.g = geom(h);
-  p.layer = layer;
-  p.nseq = nseq;
-  p.n_items = (int)items.size();
-  p.split_pages = split;
-  p.max_splits = max_splits;
-  p.grid = std::min<int>((int)items.size(), h->num_sms);
-  p.ws_meta = ws;
-  p.nsplit_off = nsplit_off;
-  p.items_off = items_off;
-  p.part_o = reinterpret_cast<float *>(static_cast<char *>(ws) + part_o_off);
-  p.part_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + part_lse_off);
-  p.q = q;
-  p.out = out;
-  p.lse = lse;
-  p.visited = reinterpret_cast<unsigned long long *>(visited);
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
-  p.scale_log2 = scale * 1.4426950408889634f;
-  SEGKV_CUDA(h, "decode launch", launch_decode(p, h->kmap, h->vmap, st));
+  if (h->pages_used + new_pages > h->cfg.num_pages) return SEGKV_ERR_OUT_OF_PAGES;
+  const StepRows step{&newk, k_new, v_new, (int)(h->pages_used + new_pages)};
+  if ((rc = decode_common(h, layer, nseq, seq_ids, pos.data(), q, softmax_scale, num_splits, out, lse, visited, ws,
+                          ws_bytes, stream, &step)))
+    return rc;
+  for (int b = 0; b < nseq; ++b) {
+    for (int k = 0; k < H; ++k) {
+      const int32_t kn = newk[(size_t)b * H + k];
+      if (kn < 0) continue;
+      const int lp = pos[b] / P;
+      const size_t row = (((size_t)layer * h->cfg.max_seqs + seq_ids[b]) * H + k) * h->max_lp;
+      h->slot_k[row + (h->cls[layer * H + k] ? lp : lp % R)] = kn;
+      h->ref[kn] = 1;
+    }
+    h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] += 1;
+  }
+  h->pages_used += new_pages;
   return SEGKV_OK;
 }
 
@@ -792,7 +872,7 @@ int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, 
     return SEGKV_ERR_INVALID_ARG;
   const int H = h->cfg.num_kv_heads;
   if (H > 1024 || n_tokens > (1 << 30)) return SEGKV_ERR_UNSUPPORTED;
-  RelocateLaunch p;
+  RelocateLaunch p{};
   p.shift = shift;
   p.q_in = q_in;
   p.q_out = q_out;
@@ -947,7 +1027,7 @@ extern "C" int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const 
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   // a copy from pageable memory has read the host buffer when it returns
   SEGKV_CUDA(h, "scratch metadata upload", cudaMemcpyAsync(scratch, host, meta_bytes, cudaMemcpyHostToDevice, st));
-  DecodeLaunch p;
+  DecodeLaunch p{};  // zeroed: fields a path does not set (the step append) stay off
   p.g = geom(h);
   p.layer = layer;
   p.nseq = nseq;
@@ -966,6 +1046,7 @@ extern "C" int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const 
   p.visited = reinterpret_cast<unsigned long long *>(visited);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.newk = nullptr;  // a plain decode: no token to append
   SEGKV_CUDA(h, "decode launch", launch_decode(p, h->kmap, h->vmap, st));
   return SEGKV_OK;
 }

@@ -25,7 +25,7 @@ EXPORTS = [
     "segkv_create", "segkv_destroy", "segkv_ring_pages", "segkv_max_lp", "segkv_seq_len", "segkv_pages_used",
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
     "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
-    "segkv_decode_attn_noalloc", "segkv_relocate_q", "segkv_fork",
+    "segkv_decode_attn_noalloc", "segkv_relocate_q", "segkv_fork", "segkv_decode_step",
 ]
 
 
@@ -75,6 +75,7 @@ def lib():
         L.segkv_decode_attn_noalloc.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P]
         L.segkv_relocate_q.argtypes = [P, I, I, P, P, P, F, I, P]
         L.segkv_fork.argtypes = [P, I, I, P]
+        L.segkv_decode_step.argtypes = [P, I, I, P, P, P, P, F, I, P, P, P, P, SZ, P]
         L.segkv_device_status.argtypes = [P, P]
         L.segkv_last_error.argtypes = [P]
         L.segkv_last_error.restype = ctypes.c_char_p
@@ -177,6 +178,13 @@ class Handle:
         return lib().segkv_decode_attn(self.h, layer, len(s), _p(s), _p(qp), _dptr(q), float(scale), int(num_splits),
                                        _dptr(out), _dptr(lse), _dptr(visited), _dptr(ws), ws_bytes, _stream(stream))
 
+    def decode_step(self, layer, seq_ids, k_new, v_new, q, scale, num_splits, out, lse, visited, ws, ws_bytes,
+                    stream=None) -> int:
+        s = _i32(seq_ids)
+        return lib().segkv_decode_step(self.h, layer, len(s), _p(s), _dptr(k_new), _dptr(v_new), _dptr(q),
+                                       float(scale), int(num_splits), _dptr(out), _dptr(lse), _dptr(visited),
+                                       _dptr(ws), ws_bytes, _stream(stream))
+
     def decode_noalloc(self, layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, stream=None) -> int:
         """segkv_decode_attn_noalloc: decode without a workspace, on the library's fixed scratch."""
         s, qp = _i32(seq_ids), _i32(q_pos)
@@ -271,6 +279,18 @@ class SegKV:
         lse = lse if lse is not None else t.empty((B, self.hq), dtype=t.float32, device=self.device)
         _check(self.handle.decode(layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, self.ws,
                                   self.ws_bytes), "segkv_decode_attn", self.handle.h)
+        return out, lse
+
+    def decode_step(self, layer: int, seq_ids, k_new, v_new, q, *, out=None, lse=None, visited=None,
+                    scale: float = 0.0, num_splits: int = 0):
+        """segkv_decode_step: appends one token per sequence (k_new, v_new [B, Hkv, D]) and
+        decodes its query q [B, Hq, D] at that position, in one decode pass."""
+        t = self.torch
+        B = len(seq_ids)
+        out = out if out is not None else t.empty((B, self.hq, self.d), dtype=t.bfloat16, device=self.device)
+        lse = lse if lse is not None else t.empty((B, self.hq), dtype=t.float32, device=self.device)
+        _check(self.handle.decode_step(layer, seq_ids, k_new, v_new, q, scale, num_splits, out, lse, visited, self.ws,
+                                       self.ws_bytes), "segkv_decode_step", self.handle.h)
         return out, lse
 
     def fork(self, src_seq: int, dst_seq: int) -> None:

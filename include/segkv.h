@@ -186,6 +186,26 @@ int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
                       void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Decode step: appends one token to every sequence and decodes its query, in one pass.
+ * For each b the token sits at position pos = segkv_seq_len(h, layer, seq_ids[b]); its K/V
+ * rows are k_new / v_new[b] (DEVICE bf16 [nseq, Hkv, D]) and its query q[b] (DEVICE bf16
+ * [nseq, Hq, D]).  Results, page tables and the allocation cursor equal those of
+ * segkv_append (num_new = 1, start_pos = pos) followed by segkv_decode_attn (q_pos = pos),
+ * bit for bit; lengths grow by one.  The append is folded into the decode kernel: the work
+ * item that holds a head's last page writes the token's rows (and a page it starts) before
+ * reading that page, so the step needs no append kernel and no second metadata upload
+ * (the per-head storage it grows: zhichai.net news item "What Happened", item 3).
+ * While a page is shared after a fork (segkv_fork), the step runs as the two calls above
+ * (the append's copy on write first); an error of the second call then leaves the token
+ * appended.
+ * Errors: INVALID_ARG (a sequence at max_seq_len, bad pointers), RING_TOO_SMALL,
+ * OUT_OF_PAGES (nothing changed), WORKSPACE, UNSUPPORTED (G > 16), CUDA.
+ */
+int segkv_decode_step(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const void *k_new, const void *v_new,
+                      const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Decode with no caller workspace and no allocation.  The pages have no counterpart to
  * this entry point; it exists for callers that cannot give the library device memory:
  * a serving engine that reserved the whole device for its own allocator at start-up, or

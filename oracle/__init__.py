@@ -50,6 +50,7 @@ def _load():
         lib.orc_append.argtypes = [P, I, I, P, P, P, P, P]
         lib.orc_fork.argtypes = [P, I, I]
         lib.orc_attention.argtypes = [P, I, I, P, P, P, P, D, P, I64, P, P, P, I]
+        lib.orc_router_scores.argtypes = [P, I, I, P, P, P, P, D, P, I]
         lib.orc_lpt_items.restype = I64
         lib.orc_lpt_items.argtypes = [I, P, P, I, P, I, I, I, P, I64]
         _lib = lib
@@ -129,6 +130,22 @@ class Oracle:
         if rc != ORC_OK:
             raise OracleError(f"orc_fork failed: {rc}")
 
+    def router_scores(self, layer: int, seq_ids: Sequence[int], q_start: Sequence[int], q_len: Sequence[int],
+                      q: np.ndarray, scale: Optional[float] = None, threads: Optional[int] = None) -> np.ndarray:
+        """Attention mass each token of the call's query range receives, summed over query
+        heads and the call's queries (fp64 [sum(q_len)], packed like q)."""
+        s, qs, ql = _i32(seq_ids), _i32(q_start), _i32(q_len)
+        qq = np.ascontiguousarray(q, dtype=np.uint16)
+        T = int(ql.sum())
+        assert qq.size == T * self.hq * self.d
+        out = np.zeros(max(T, 1))
+        sc = float(scale) if scale is not None else 1.0 / np.sqrt(self.d)
+        rc = self.lib.orc_router_scores(self.h, layer, len(s), _ptr(s), _ptr(qs), _ptr(ql), _ptr(qq), sc, _ptr(out),
+                                        threads or host_threads())
+        if rc:
+            raise OracleError(f"orc_router_scores failed with {rc}")
+        return out[:T]
+
     def attention(self, layer: int, seq_ids: Sequence[int], q_start: Sequence[int], q_len: Sequence[int],
                   q: np.ndarray, scale: Optional[float] = None, rows: Optional[np.ndarray] = None,
                   threads: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
@@ -149,6 +166,22 @@ class Oracle:
         if rc:
             raise OracleError(f"orc_attention failed with {rc}")
         return out, lse, counts
+
+
+def topk_rows(scores: np.ndarray, q_len: Sequence[int], k: Sequence[int]) -> np.ndarray:
+    """Top-k routing over packed per-token scores (reading: the k highest scores of each
+    sequence, equal scores by lower position first; rows returned ascending, sequences in
+    call order).  Returns int32 packed rows."""
+    out, off = [], 0
+    for n, kk in zip(q_len, k):
+        n, kk = int(n), int(kk)
+        if not 0 <= kk <= n:
+            raise OracleError("k outside [0, q_len]")
+        s = np.asarray(scores[off:off + n])
+        order = np.lexsort((np.arange(n), -s))  # score descending, then position ascending
+        out.append(np.sort(order[:kk]) + off)
+        off += n
+    return np.concatenate(out).astype(np.int32) if out else np.zeros(0, np.int32)
 
 
 def lpt_items(q_start, q_len, classes_layer, window: int, tile_pos: int, bn: int) -> np.ndarray:

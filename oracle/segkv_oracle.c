@@ -402,3 +402,127 @@ int64_t orc_lpt_items(int nseq, const int32_t *q_start, const int32_t *q_len, in
   free(it);
   return n;
 }
+
+/*
+ * Attention as a router (zhichai.net news item "What Happened", item 2 and its body: dense
+ * FFN only on the top-k tokens by attention score, an identity path for the rest;
+ * hysenlabs.com write-up, "The Three Core Mechanisms in Detail", second mechanism:
+ * token-level importance scores decide which tokens enter the FFN).  The pages do not
+ * define the score; the reading taken here is the attention mass a token receives:
+ *   score[j] = sum over query heads h and over the call's queries i of sequence b that
+ *              see j of  softmax_h(i)[j] = exp(scale q_{i,h}.k_j - lse_{i,h}),
+ * for every token j of the call's own query range (the tokens whose FFN rows are being
+ * routed).  Each query row is computed as in one_row (explicit visibility row, fp64
+ * scores, its own lse); its weights are then added to the scores of the keys in range.
+ * scores: fp64 [sum(q_len)], packed like q.
+ */
+typedef struct {
+  job_t base;
+  double **acc; /* per worker: fp64 [sum(q_len)] */
+  int next_worker;
+} router_job_t;
+
+static int router_row(job_t *j, int64_t r, uint8_t *vis, double *x, double *acc) {
+  const orc_t *o = j->o;
+  const int D = o->d, G = o->hq / o->hkv;
+  const int64_t tok = r / o->hq;
+  const int hqi = (int)(r % o->hq);
+  int b = 0;
+  while (b + 1 < j->nseq && j->q_off[b + 1] <= tok) ++b;
+  const int seq = j->seq_ids[b];
+  const int p = j->q_start[b] + (int)(tok - j->q_off[b]);
+  const int kvh = hqi / G;
+  const int global = o->cls[j->layer * o->hkv + kvh];
+  const int L = o->len[(size_t)j->layer * o->max_seqs + seq];
+  if (p >= L) return ORC_ERR_ARG;
+  for (int k = 0; k < L; ++k) vis[k] = global ? (k <= p) : (k <= p && k > p - o->window);
+  const uint16_t *qr = j->q + (size_t)r * D;
+  double m = -INFINITY;
+  for (int k = 0; k < L; ++k) {
+    if (!vis[k]) continue;
+    const uint16_t *kr = read_token(o, o->kpool, j->layer, seq, kvh, k);
+    if (!kr) return ORC_ERR_NOT_RESIDENT;
+    double s = 0.0;
+    for (int dd = 0; dd < D; ++dd) s += bf16_to_double(qr[dd]) * bf16_to_double(kr[dd]);
+    x[k] = j->scale * s;
+    if (x[k] > m) m = x[k];
+  }
+  double z = 0.0;
+  for (int k = 0; k < L; ++k)
+    if (vis[k]) z += exp(x[k] - m);
+  const double lse = m + log(z);
+  const int k_lo = j->q_start[b], k_hi = j->q_start[b] + j->q_len[b] - 1;
+  for (int k = k_lo; k <= k_hi && k < L; ++k)
+    if (vis[k]) acc[j->q_off[b] + (k - k_lo)] += exp(x[k] - lse);
+  return ORC_OK;
+}
+
+static void *router_worker(void *arg) {
+  router_job_t *rj = (router_job_t *)arg;
+  job_t *j = &rj->base;
+  pthread_mutex_lock(&j->mu);
+  double *acc = rj->acc[rj->next_worker++];
+  pthread_mutex_unlock(&j->mu);
+  const int cap = j->o->max_seq_len;
+  uint8_t *vis = (uint8_t *)malloc((size_t)cap);
+  double *x = (double *)malloc(sizeof(double) * (size_t)cap);
+  for (;;) {
+    pthread_mutex_lock(&j->mu);
+    int64_t i = j->next;
+    j->next += 16;
+    int err = j->err;
+    pthread_mutex_unlock(&j->mu);
+    if (i >= j->nrows || err) break;
+    int64_t e = i + 16 < j->nrows ? i + 16 : j->nrows;
+    for (; i < e; ++i) {
+      int rc = router_row(j, i, vis, x, acc);
+      if (rc) {
+        pthread_mutex_lock(&j->mu);
+        j->err = rc;
+        pthread_mutex_unlock(&j->mu);
+        break;
+      }
+    }
+  }
+  free(vis);
+  free(x);
+  return NULL;
+}
+
+int orc_router_scores(const orc_t *o, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start,
+                      const int32_t *q_len, const uint16_t *q, double scale, double *scores, int nthreads) {
+  if (layer < 0 || layer >= o->layers || nseq < 1) return ORC_ERR_ARG;
+  int32_t *q_off = (int32_t *)malloc(sizeof(int32_t) * (size_t)(nseq + 1));
+  q_off[0] = 0;
+  for (int b = 0; b < nseq; ++b) {
+    if (seq_ids[b] < 0 || seq_ids[b] >= o->max_seqs || q_len[b] < 0 || q_start[b] < 0) {
+      free(q_off);
+      return ORC_ERR_ARG;
+    }
+    q_off[b + 1] = q_off[b] + q_len[b];
+  }
+  const int64_t T = q_off[nseq];
+  if (nthreads < 1) nthreads = 1;
+  router_job_t rj;
+  memset(&rj, 0, sizeof(rj));
+  job_t *j = &rj.base;
+  j->o = o; j->layer = layer; j->nseq = nseq; j->seq_ids = seq_ids; j->q_start = q_start; j->q_len = q_len;
+  j->q_off = q_off; j->q = q; j->scale = scale; j->nrows = T * o->hq;
+  pthread_mutex_init(&j->mu, NULL);
+  rj.acc = (double **)malloc(sizeof(double *) * (size_t)nthreads);
+  for (int t = 0; t < nthreads; ++t) rj.acc[t] = (double *)calloc((size_t)(T > 0 ? T : 1), sizeof(double));
+  pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  for (int t = 0; t < nthreads; ++t) pthread_create(&th[t], NULL, router_worker, &rj);
+  for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+  free(th);
+  pthread_mutex_destroy(&j->mu);
+  for (int64_t i = 0; i < T; ++i) {
+    double s = 0.0;
+    for (int t = 0; t < nthreads; ++t) s += rj.acc[t][i];
+    scores[i] = s;
+  }
+  for (int t = 0; t < nthreads; ++t) free(rj.acc[t]);
+  free(rj.acc);
+  free(q_off);
+  return j->err;
+}

@@ -41,3 +41,24 @@ def dense_masked_attention(q_bits, k_bits, v_bits, q_pos, classes, window, scale
         lse[:, h] = (m + np.log(z))[:, 0]
     counts = mask.sum(axis=(1, 2))
     return out, lse, counts
+
+
+def dense_received_attention(q_bits, k_bits, q_pos, key_lo, key_hi, classes, window, scale):
+    """Attention mass received by the keys at positions [key_lo, key_hi): for each, the sum
+    over query heads and query rows of the dense masked softmax weight.  q_bits [Lq, Hq, D]
+    at absolute positions q_pos; k_bits [L, Hkv, D] at positions 0..L-1.  fp64 [key_hi - key_lo]."""
+    q = bf16_bits_to_f32(q_bits).astype(np.float64)
+    k = bf16_bits_to_f32(k_bits).astype(np.float64)
+    Lq, Hq, _ = q.shape
+    L, Hkv, _ = k.shape
+    G = Hq // Hkv
+    key = np.arange(L)[None, :]
+    qp = np.asarray(q_pos)[:, None]
+    total = np.zeros(L)
+    for h in range(Hq):
+        kv = h // G
+        mask = key <= qp if classes[kv] else (key <= qp) & (key > qp - window)
+        s = np.where(mask, scale * q[:, h, :] @ k[:, kv, :].T, -np.inf)
+        e = np.exp(s - s.max(axis=1, keepdims=True))
+        total += (e / e.sum(axis=1, keepdims=True)).sum(axis=0)
+    return total[key_lo:key_hi]

@@ -388,6 +388,35 @@ def main():
                 "roofline": {"bound": "hbm", "achieved": rel_bytes / (t_rel * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                              "unit": "GB/s", "frac": rel_bytes / (t_rel * 1e-3) / 1e9 / pk["hbm_gbs"], "traffic": None,
                              "kernel": "relocate_q_kernel (events around segkv_relocate_q)"}}
+    # ------------------------------------------------------------------ attention as a router
+    # segkv_router_topk on the same queries and the last prefill's lse: every token's received
+    # attention mass and the top quarter of the tokens.  One exponential per visible pair on
+    # the MUFU bounds it (16 per clock per SM).
+    k_top = [L // 4]
+    for _ in range(args.warmup):
+        kv.router_topk(0, [0], [0], [L], q_d, lse, k_top)
+    evt = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(args.steps, 50))]
+    for e in evt:
+        flush.fill_(2)
+        e[0].record(stream)
+        kv.router_topk(0, [0], [0], [L], q_d, lse, k_top)
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the router benchmark")
+    t_rt = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evt) / len(evt))
+    pairs = visible_pairs(w)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    max_mhz = float((clocks or {}).get("sm_max_mhz") or 1965.0)  # the GPU's maximum SM clock (nvidia-smi)
+    mufu_peak = 16 * sms * max_mhz * 1e6 / 1e9  # G exponentials per second at that clock
+    router = {"metric": "router visible pairs/s", "value": world * pairs / (t_rt * 1e-3) / 1e9, "unit": "Gpair/s",
+              "ms_per_call": t_rt, "pairs_per_call": pairs, "k": k_top[0],
+              "step": "segkv_router_topk: received attention mass of 8192 tokens (32 query heads) + top 2048",
+              "roofline": {"bound": "alu", "achieved": pairs / (t_rt * 1e-3) / 1e9, "peak": mufu_peak,
+                           "unit": "Gexp/s", "frac": pairs / (t_rt * 1e-3) / 1e9 / mufu_peak, "traffic": None,
+                           "peak_source": f"MUFU ex2: 16 per clock per SM x {sms} SMs x {max_mhz:.0f} MHz",
+                           "kernel": "router_kernel<128> + topk_kernel (events around segkv_router_topk)"},
+              "gpu_launches": 2 * len(evt)}
     del kv, flush, q_rel
     torch.cuda.empty_cache()
 
@@ -415,6 +444,7 @@ def main():
         "clocks": clocks,
     }
     line["relocate"] = relocate
+    line["router"] = router
     line["fork"] = bench_fork(args, torch, dev, stream, max_over_ranks, world, pk)
     if decode is not None:
         line["decode"] = decode

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libsegkv.so")
-SOURCES = ["segkv_runtime.cu", "storage.cu", "prefill_sm100.cu", "decode.cu", "rope.cu"]
+SOURCES = ["segkv_runtime.cu", "storage.cu", "prefill_sm100.cu", "decode.cu", "rope.cu", "router_sm100.cu"]
 HEADERS = ["internal.h", "device_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -29,6 +29,8 @@ constexpr int kPrefillItemRows = 256;  // rows of one prefill work item (two que
 constexpr int kPrefillKeyTile = 128;   // keys of a prefill key tile
 constexpr int kDecodeStageKeys = 64;   // keys of a decode pipeline stage
 constexpr int kMaxSplits = 32;         // most splits one decode head is cut into
+constexpr int kRouterKeys = 128;       // keys of a router key tile
+constexpr int kRouterMaxChunks = 8;    // most chunks one router key tile is cut into
 constexpr int kStagingSlots = 4;
 constexpr int kMaxChunks = 32;         // most chunks one prefill item is cut into
 
@@ -315,6 +317,12 @@ size_t prefill_part_bytes(int head_dim) {
   return (size_t)kMaxPartSlots * 2 * 128 * ((size_t)head_dim + 1) * 4;
 }
 
+// Router workspace: header, sequences, items, per-sequence top-k rows, then the partials.
+size_t router_meta_bytes(int nseq, size_t n_items) {
+  return align_up(align_up(kHeaderBytes + sizeof(RouterSeq) * nseq, 16) + 16 * n_items + 16 * (size_t)nseq, 256);
+}
+size_t router_part_bytes(int chunks, int hkv, long long n_tokens) { return 4 * (size_t)chunks * hkv * n_tokens; }
+
 // The token of a decode step, appended by the decode kernel itself: newk[b * hkv + h] =
 // free-list entry of a page the token starts (-1: written in place), K/V rows on the device.
 struct StepRows {
@@ -506,12 +514,16 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
   const size_t pre = prefill_meta_bytes(max_batch, H * ((size_t)ceil_div(max_tokens, tile_pos) + max_batch) +
                                                       kMaxPartSlots, kMaxPartSlots) +
                      prefill_part_bytes((int)D);
-  const size_t dec_meta = align_up(kHeaderBytes + sizeof(DecodeSeq) * max_batch + 4 * max_batch * H +
+  // decode: split counts and (decode step) new page ids per (sequence, head), then the items
+  const size_t dec_meta = align_up(kHeaderBytes + sizeof(DecodeSeq) * max_batch + 8 * max_batch * H +
                                        8 * max_batch * H * kMaxSplits + 16,
                                    256);
   const size_t dec = dec_meta + align_up(4 * (size_t)max_batch * Hq * kMaxSplits * D, 256) +
                      4 * (size_t)max_batch * Hq * kMaxSplits;
-  return align_up(std::max(app, std::max(pre, dec)), 256);
+  const size_t rt = router_meta_bytes(max_batch, H * ((size_t)max_tokens / kRouterKeys + 2 * max_batch) *
+                                                     kRouterMaxChunks) +
+                    router_part_bytes(kRouterMaxChunks, (int)H, max_tokens);
+  return align_up(std::max(std::max(app, rt), std::max(pre, dec)), 256);
 }
 
 int segkv_reset(segkv_t *h, void *stream) {
@@ -858,6 +870,134 @@ int segkv_decode_step(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
     h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] += 1;
   }
   h->pages_used += new_pages;
+  return SEGKV_OK;
+}
+
+int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                      const int32_t *q_len, const void *q, const float *lse, float softmax_scale, const int32_t *k,
+                      float *scores, int32_t *rows_out, void *ws, size_t ws_bytes, void *stream) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  int rc = check_seqs(h, layer, nseq, seq_ids);
+  if (rc) return rc;
+  if (!q_start_pos || !q_len || !k) return SEGKV_ERR_INVALID_ARG;
+  const int G = h->G, P = h->cfg.page_size, H = h->cfg.num_kv_heads, W = h->cfg.window;
+  if (G > 16 || (G & (G - 1)) != 0) return SEGKV_ERR_UNSUPPORTED;
+  const bool has_local = layer_has_local(h, layer);
+  long long tq = 0, tk = 0;
+  for (int b = 0; b < nseq; ++b) {
+    const int len = h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]];
+    if (q_len[b] < 0 || q_start_pos[b] < 0 || (long long)q_start_pos[b] + q_len[b] > len) return SEGKV_ERR_INVALID_ARG;
+    if (k[b] < 0 || k[b] > q_len[b]) return SEGKV_ERR_INVALID_ARG;
+    // every scored token must still be stored in every local head
+    if (q_len[b] > 0 && has_local && q_start_pos[b] / P < (len - 1) / P - h->ring + 1) return SEGKV_ERR_RING_TOO_SMALL;
+    tq += q_len[b];
+    tk += k[b];
+  }
+  if (tq == 0) return SEGKV_OK;
+  if (tq > (1LL << 30)) return SEGKV_ERR_UNSUPPORTED;
+  if (!q || !lse || !scores || !aligned(q, 16) || !aligned(lse, 4) || !aligned(scores, 4)) return SEGKV_ERR_INVALID_ARG;
+  if (tk > 0 && (!rows_out || !aligned(rows_out, 4))) return SEGKV_ERR_INVALID_ARG;
+  if ((rc = ensure_device_state(h))) return rc;
+  // items: (sequence, KV head, key tile, chunk of query tiles), longest first
+  const int tile_pos = kRouterKeys / G;
+  struct Span {
+    int b, kt;
+  };
+  std::vector<Span> spans;
+  long long total_tiles = 0;
+  for (int b = 0; b < nseq; ++b) {
+    if (q_len[b] == 0) continue;
+    const int qs = q_start_pos[b], qe = qs + q_len[b];
+    for (int kt = qs / kRouterKeys; kt <= (qe - 1) / kRouterKeys; ++kt) spans.push_back({b, kt});
+  }
+  std::vector<int4> items;
+  std::vector<int32_t> cost;
+  int max_n = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    const long long share = std::max<long long>(1, (total_tiles + 2LL * h->num_sms - 1) / (2LL * h->num_sms));
+    for (const Span &sp : spans)
+      for (int hh = 0; hh < H; ++hh) {
+        const bool global = h->cls[layer * H + hh] != 0;
+        const int qs = q_start_pos[sp.b], qe = qs + q_len[sp.b];
+        const int k_lo = std::max(sp.kt * kRouterKeys, qs), k_hi = std::min(sp.kt * kRouterKeys + kRouterKeys - 1, qe - 1);
+        const int q_hi = global ? qe - 1 : std::min(qe - 1, k_hi + W - 1);
+        const int n = ceil_div(q_hi - k_lo + 1, tile_pos);
+        if (pass == 0) {
+          total_tiles += n;
+          max_n = std::max(max_n, n);
+          continue;
+        }
+        const int C = (int)std::min<long long>(kRouterMaxChunks, std::max<long long>(1, (n + share - 1) / share));
+        for (int c = 0; c < C; ++c) {
+          const int t0 = (int)((long long)n * c / C), t1 = (int)((long long)n * (c + 1) / C);
+          if (t1 <= t0) continue;
+          items.push_back(make_int4(sp.b, (int)make_item_w1(global, hh, sp.kt), t0, (c << 20) | (t1 - t0)));
+        }
+      }
+  }
+  int chunks = 1;
+  for (const int4 &it : items) chunks = std::max(chunks, ((int)((uint32_t)it.w >> 20)) + 1);
+  {
+    std::vector<size_t> order(items.size());
+    for (size_t i = 0; i < order.size(); ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](size_t x, size_t y) {
+      return (items[x].w & 0xFFFFF) > (items[y].w & 0xFFFFF);
+    });
+    std::vector<int4> sorted(items.size());
+    for (size_t i = 0; i < order.size(); ++i) sorted[i] = items[order[i]];
+    items.swap(sorted);
+  }
+  const size_t items_off = align_up(kHeaderBytes + sizeof(RouterSeq) * nseq, 16);
+  const size_t topk_off = items_off + 16 * items.size();
+  const size_t bytes = topk_off + 16 * (size_t)nseq;
+  const size_t part_off = router_meta_bytes(nseq, items.size());
+  const size_t need = part_off + router_part_bytes(chunks, H, tq);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEGKV_ERR_WORKSPACE;
+  const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads;
+  CUtensorMap qmap;
+  if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, G, tile_pos)) {
+    h->last_error = "query tensor map encode failed";
+    return SEGKV_ERR_CUDA;
+  }
+  void *host = nullptr;
+  if ((rc = staging(h, bytes, &host))) return rc;
+  std::memset(host, 0, items_off);
+  RouterSeq *rs = reinterpret_cast<RouterSeq *>(static_cast<char *>(host) + kHeaderBytes);
+  int4 *tm = reinterpret_cast<int4 *>(static_cast<char *>(host) + topk_off);
+  int row0 = 0, out0 = 0;
+  for (int b = 0; b < nseq; ++b) {
+    rs[b] = RouterSeq{seq_ids[b], q_start_pos[b], q_len[b], row0, h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]],
+                      0, 0, 0};
+    tm[b] = make_int4(row0, q_len[b], k[b], out0);
+    row0 += q_len[b];
+    out0 += k[b];
+  }
+  if (!items.empty())
+    std::memcpy(static_cast<char *>(host) + items_off, items.data(), 16 * items.size());
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = upload(h, ws, bytes, st))) return rc;
+  float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + part_off);
+  SEGKV_CUDA(h, "router partials clear", cudaMemsetAsync(part, 0, router_part_bytes(chunks, H, tq), st));
+  RouterLaunch p{};
+  p.g = geom(h);
+  p.layer = layer;
+  p.nseq = nseq;
+  p.n_items = (int)items.size();
+  p.tile_pos = tile_pos;
+  p.g_shift = 0;
+  while ((1 << p.g_shift) < G) ++p.g_shift;
+  p.grid = std::min<int>((int)items.size(), h->num_sms);
+  p.n_tokens = (int)tq;
+  p.ws_meta = ws;
+  p.items_off = (int)items_off;
+  p.lse = lse;
+  p.part = part;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (p.n_items > 0) SEGKV_CUDA(h, "router launch", launch_router(p, qmap, h->kmap, st));
+  SEGKV_CUDA(h, "top-k launch",
+             launch_topk(part, chunks, H, (int)tq, reinterpret_cast<const int4 *>(static_cast<char *>(ws) + topk_off),
+                         nseq, scores, rows_out, st));
   return SEGKV_OK;
 }
 

@@ -26,6 +26,7 @@ EXPORTS = [
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
     "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
     "segkv_decode_attn_noalloc", "segkv_relocate_q", "segkv_fork", "segkv_decode_step",
+    "segkv_router_topk",
 ]
 
 
@@ -75,6 +76,7 @@ def lib():
         L.segkv_decode_attn_noalloc.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P]
         L.segkv_relocate_q.argtypes = [P, I, I, P, P, P, F, I, P]
         L.segkv_fork.argtypes = [P, I, I, P]
+        L.segkv_router_topk.argtypes = [P, I, I, P, P, P, P, P, F, P, P, P, P, SZ, P]
         L.segkv_decode_step.argtypes = [P, I, I, P, P, P, P, F, I, P, P, P, P, SZ, P]
         L.segkv_device_status.argtypes = [P, P]
         L.segkv_last_error.argtypes = [P]
@@ -185,6 +187,13 @@ class Handle:
                                        float(scale), int(num_splits), _dptr(out), _dptr(lse), _dptr(visited),
                                        _dptr(ws), ws_bytes, _stream(stream))
 
+    def router_topk(self, layer, seq_ids, q_start, q_len, q, lse, scale, k, scores, rows_out, ws, ws_bytes,
+                    stream=None) -> int:
+        s, qs, ql, kk = _i32(seq_ids), _i32(q_start), _i32(q_len), _i32(k)
+        return lib().segkv_router_topk(self.h, layer, len(s), _p(s), _p(qs), _p(ql), _dptr(q), _dptr(lse),
+                                       float(scale), _p(kk), _dptr(scores), _dptr(rows_out), _dptr(ws), ws_bytes,
+                                       _stream(stream))
+
     def decode_noalloc(self, layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, stream=None) -> int:
         """segkv_decode_attn_noalloc: decode without a workspace, on the library's fixed scratch."""
         s, qp = _i32(seq_ids), _i32(q_pos)
@@ -292,6 +301,18 @@ class SegKV:
         _check(self.handle.decode_step(layer, seq_ids, k_new, v_new, q, scale, num_splits, out, lse, visited, self.ws,
                                        self.ws_bytes), "segkv_decode_step", self.handle.h)
         return out, lse
+
+    def router_topk(self, layer: int, seq_ids, q_start, q_len, q, lse, k, *, scores=None, rows=None,
+                    scale: float = 0.0):
+        """segkv_router_topk: each token's received attention mass (fp32 [sum(q_len)]) and the
+        packed rows of the k[b] highest-scoring tokens of every sequence (int32 [sum(k)])."""
+        t = self.torch
+        T, K = int(sum(q_len)), int(sum(k))
+        scores = scores if scores is not None else t.empty((T,), dtype=t.float32, device=self.device)
+        rows = rows if rows is not None else t.empty((max(K, 1),), dtype=t.int32, device=self.device)
+        _check(self.handle.router_topk(layer, seq_ids, q_start, q_len, q, lse, scale, k, scores, rows, self.ws,
+                                       self.ws_bytes), "segkv_router_topk", self.handle.h)
+        return scores, rows[:K]
 
     def fork(self, src_seq: int, dst_seq: int) -> None:
         """segkv_fork: dst_seq (empty) shares src_seq's pages; appends copy shared pages first."""

@@ -206,6 +206,29 @@ int segkv_decode_step(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
                       void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Attention as a router (zhichai.net news item "What Happened", item 2: the dense FFN runs
+ * only on the top-k tokens by attention score, the rest take an identity path; hysenlabs.com
+ * write-up, "The Three Core Mechanisms in Detail", second mechanism: token-level importance
+ * scores).  The pages leave the score undefined; here a token's score is the attention mass
+ * it receives from the call's queries:
+ *   scores[j] = sum over query heads h and queries i of the call that see token j of
+ *               exp(scale * q_{i,h} . k_j - lse_{i,h})        (fp32, >= 0),
+ * for every token j of the call's query range (the FFN rows being routed); lse is the
+ * output of segkv_prefill_attn for the same queries (DEVICE fp32 [sum(q_len), Hq]), q the
+ * same queries (DEVICE bf16 [sum(q_len), Hq, D]).  scores: DEVICE fp32 [sum(q_len)], packed
+ * like q.  Then, per sequence, the k[b] (HOST int32 [nseq], 0 <= k[b] <= q_len[b]) highest
+ * scores, equal scores by lower position first: rows_out (DEVICE int32 [sum(k)]) receives
+ * their packed rows, ascending within a sequence, sequences in call order.  The scores do
+ * not depend on the schedule (each key's partial sums have their own slot and are added in
+ * a fixed order).  Requires G = Hq / Hkv a power of two <= 16.
+ * Errors: INVALID_ARG (ranges, k out of range, alignment), RING_TOO_SMALL (a scored token
+ * is no longer stored in a local head), WORKSPACE, UNSUPPORTED, CUDA.
+ */
+int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                      const int32_t *q_len, const void *q, const float *lse, float softmax_scale, const int32_t *k,
+                      float *scores, int32_t *rows_out, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Decode with no caller workspace and no allocation.  The pages have no counterpart to
  * this entry point; it exists for callers that cannot give the library device memory:
  * a serving engine that reserved the whole device for its own allocator at start-up, or

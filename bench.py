@@ -393,13 +393,15 @@ def main():
     # attention mass and the top quarter of the tokens.  One exponential per visible pair on
     # the MUFU bounds it (16 per clock per SM).
     k_top = [L // 4]
+    rt_scores = torch.empty((L,), dtype=torch.float32, device=dev)
+    rt_rows = torch.empty((L // 4,), dtype=torch.int32, device=dev)
     for _ in range(args.warmup):
-        kv.router_topk(0, [0], [0], [L], q_d, lse, k_top)
+        kv.router_topk(0, [0], [0], [L], q_d, lse, k_top, scores=rt_scores, rows=rt_rows)
     evt = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(args.steps, 50))]
     for e in evt:
         flush.fill_(2)
         e[0].record(stream)
-        kv.router_topk(0, [0], [0], [L], q_d, lse, k_top)
+        kv.router_topk(0, [0], [0], [L], q_d, lse, k_top, scores=rt_scores, rows=rt_rows)
         e[1].record(stream)
     torch.cuda.synchronize()
     if kv.device_status() != 0:
@@ -415,8 +417,8 @@ def main():
               "roofline": {"bound": "alu", "achieved": pairs / (t_rt * 1e-3) / 1e9, "peak": mufu_peak,
                            "unit": "Gexp/s", "frac": pairs / (t_rt * 1e-3) / 1e9 / mufu_peak, "traffic": None,
                            "peak_source": f"MUFU ex2: 16 per clock per SM x {sms} SMs x {max_mhz:.0f} MHz",
-                           "kernel": "router_kernel<128> + topk_kernel (events around segkv_router_topk)"},
-              "gpu_launches": 2 * len(evt)}
+                           "kernel": "router_kernel<128> + score_sum_kernel + topk_kernel (events around segkv_router_topk)"},
+              "gpu_launches": 3 * len(evt)}
     del kv, flush, q_rel
     torch.cuda.empty_cache()
 

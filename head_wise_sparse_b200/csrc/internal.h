@@ -108,6 +108,9 @@ int decode_smem_bytes(int head_dim);
 // call, w1 = (global << 31) | (kv_head << 20) | key tile (128 absolute positions), w2 = first
 // query tile of the item, w3 = (chunk << 20) | number of query tiles.  Query tile t of key
 // tile kt holds tile_pos positions from max(kt * 128, q_start) + t * tile_pos, all G heads.
+// Reducing warps of the router kernel per TMEM lane quadrant; each sums 128 / groups of
+// the 128 query columns, and each (chunk, column group) has its own partial slot.
+constexpr int kRouterColGroups = 4;
 struct RouterSeq {
   int32_t seq_id, q_start, q_len, q_row0;
   int32_t kv_len, pad0, pad1, pad2;
@@ -118,17 +121,18 @@ struct RouterLaunch {
   const void *ws_meta;  // header + RouterSeq[nseq] + items (int4)
   int items_off;
   const float *lse;     // [n_tokens, hq] natural-log lse of the queries
-  float *part;          // [chunks][hkv][n_tokens]: each item's received mass per key
+  float *part;          // [chunks][column groups][hkv][n_tokens]: received mass per key
   float scale_log2;
 };
 cudaError_t launch_router(const RouterLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
                           cudaStream_t st);
 int router_smem_bytes(int head_dim);
 
-// Top-k per sequence over scores[t] = sum over chunks and KV heads of part; one CTA per
-// sequence.  topk_meta: int4 per sequence (q_row0, q_len, k, first output row).
+// scores[t] = sum over partial slots and KV heads of part (one thread per token), then the
+// top-k per sequence (one CTA per sequence).  topk_meta: int4 per sequence (q_row0, q_len,
+// k, first output row).
 cudaError_t launch_topk(const float *part, int chunks, int hkv, int n_tokens, const int4 *topk_meta, int nseq,
-                        float *scores, int32_t *rows_out, cudaStream_t st);
+                        int max_len, float *scores, int32_t *rows_out, cudaStream_t st);
 
 struct RelocateLaunch {
   const int32_t *shift;  // DEVICE [n_tokens]: the position offset of each packed token

@@ -15,19 +15,26 @@
 // consecutive positions -- the B operand (N = 128).  Each thread of the four reducing warps
 // owns one key and sums its TMEM row of weights in registers: no cross-thread reduction.
 // One exponential per visible pair bounds the kernel; the dot products ride the tensor core.
-// CTA of 192 threads:
-//   warp 0      producer: the key tile once per item (pages resolved through the head's
-//               page table), then the item's query tiles through a 4-deep ring, each with
-//               the 128 lse values of its columns (log2 domain; +inf marks a column past
-//               the sequence's queries, whose weight is then exactly 0)
+// CTA of 640 threads (96 registers each):
+//   warp 0      producer: the key tile once per item into one of two buffers (pages resolved
+//               through the head's page table), then the item's query tiles through a
+//               4-deep ring, each with the 128 negated lse values of its columns (log2
+//               domain, loaded one tile ahead; -inf marks a column past the sequence's
+//               queries, whose weight is then exactly 0)
 //   warp 1      lane 0 issues the MMAs into two 128-column S buffers in TMEM
-//   warps 2..5  one key row per thread; a key's sums over the item go to the item's
-//               partial slot [chunk][KV head][token], so the result does not depend on
-//               the schedule
-// topk_kernel.  One CTA per sequence: adds the partials in a fixed order, writes the
-// scores, finds the k-th largest by a radix select over the float bits (scores are >= 0,
-// so their bit patterns are ordered like their values), and writes the selected rows in
-// ascending order -- equal scores at the threshold by lower position -- with block scans.
+//   warps 2, 3  idle
+//   warps 4..19 four warps per TMEM lane quadrant, each summing 32 of the 128 columns of
+//               its 32 keys (one key per thread); a key's sums over the item go to the
+//               item's partial slot [chunk][column group][KV head][token], so the result
+//               does not depend on the schedule
+// score_sum_kernel.  One thread per token adds its partials in a fixed order (slot, then
+// KV head) and writes the score.
+// topk_kernel.  One CTA per sequence finds the k-th largest score by a radix select over
+// the float bits (scores are >= 0, so their bit patterns are ordered like their values),
+// and writes the selected rows in ascending order -- equal scores at the threshold by lower
+// position -- with block scans.
+#include <algorithm>
+
 #include "device_common.cuh"
 
 namespace skv {
@@ -37,20 +44,31 @@ namespace {
 constexpr int kRKeys = 128;     // keys of a tile (M of the MMA, TMEM lanes)
 constexpr int kRCols = 128;     // query rows of a tile (N of the MMA)
 constexpr int kRStages = 4;     // query-tile ring depth
-constexpr int kRThreads = 192;
+constexpr int kRReducers = 4 * kRouterColGroups;  // reducing warps: kRouterColGroups per lane quadrant
+constexpr int kRGroupCols = kRCols / kRouterColGroups;
+constexpr int kRThreads = 128 + 32 * kRReducers;
+static_assert(kRGroupCols % 32 == 0, "whole 32-column TMEM loads");
+// With two groups (384 threads, 168 registers a thread at launch) the first warpgroup drops
+// to 104 registers (the producer needs that many without spilling) and the two reducing
+// warpgroups rise to 200: 128 x 104 + 256 x 200 = 64512 = 384 x 168.
+constexpr bool kRSplitRegs = kRouterColGroups == 2;
+constexpr int kRRegsLaunch = (65536 / kRThreads) / 8 * 8;
+constexpr int kRRegsLow = 104, kRRegsHigh = (kRRegsLaunch * kRThreads - 128 * kRRegsLow) / 256 / 8 * 8;
+static_assert(!kRSplitRegs || (kRRegsHigh == 200 && 128 * kRRegsLow + 256 * kRRegsHigh <= kRRegsLaunch * kRThreads),
+              "register split exceeds the launch total");
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct RSmem {
-  static constexpr int kTileBytes = kRKeys * D * 2;  // the K tile and each Q tile (128 rows)
-  static constexpr int kQOff = kTileBytes;
+  static constexpr int kTileBytes = kRKeys * D * 2;  // a K tile and each Q tile (128 rows)
+  static constexpr int kQOff = 2 * kTileBytes;
   static constexpr int kLseOff = kQOff + kRStages * kTileBytes;
   static constexpr int kBarOff = kLseOff + kRStages * kRCols * 4;
   static constexpr int kBytes = 1024 + kBarOff + 512;
 };
 
 struct RBars {
-  uint64_t k_full, k_empty;
+  uint64_t k_full[2], k_empty[2];
   uint64_t q_full[kRStages], q_empty[kRStages], l_full[kRStages], l_empty[kRStages];
   uint64_t s_full[2], s_empty[2];
   uint64_t mma_done;
@@ -115,7 +133,8 @@ __device__ __forceinline__ void router_producer(const CUtensorMap &qmap, const C
     }
     if (idx < 0) break;
     const RItem it = decode_ritem(p, seqs, items, idx);
-    if (!(ok = warp_wait(&bar->k_empty, (i & 1) ^ 1, abort_flag, state))) break;
+    const int kb = i & 1;  // K buffer of this item
+    if (!(ok = warp_wait(&bar->k_empty[kb], ((i >> 1) & 1) ^ 1, abort_flag, state))) break;
     // the key tile: pages kt * PPT .. kt * PPT + PPT - 1, one per lane; pages not stored load zeros
     const long long row_base = (((long long)p.layer * p.g.max_seqs + it.seq_id) * p.g.hkv + it.h) * p.g.max_lp;
     const int last_lp = (it.kv_len - 1) / P;
@@ -129,27 +148,48 @@ __device__ __forceinline__ void router_producer(const CUtensorMap &qmap, const C
         else if (lp * P + P - 1 >= it.q_start && lp * P < it.q_end) set_error(state, kErrDeviceBounds);
       }
     }
-    if (lane == 0) mbar_expect_tx(&bar->k_full, S::kTileBytes);
+    if (lane == 0) mbar_expect_tx(&bar->k_full[kb], S::kTileBytes);
     for (int j = 0; j < PPT; ++j) {
       const int phys = __shfl_sync(0xffffffffu, pid, j);
       if (lane == 0)
         for (int hh = 0; hh < D / 64; ++hh)
-          tma_load_3d(k_s + hh * kRKeys * 128 + j * P * 128, &kmap, &bar->k_full, hh * 64, 0, phys);
+          tma_load_3d(k_s + kb * S::kTileBytes + hh * kRKeys * 128 + j * P * 128, &kmap, &bar->k_full[kb], hh * 64,
+                      0, phys);
     }
     ++k_loads;
+    // the negated log2-domain lse of column lane + 32 j of query tile t
+    auto neg_lse = [&](int t, int j) -> float {
+      const int qa = it.k_lo + (it.t0 + t) * p.tile_pos;
+      const int col = lane + 32 * j;
+      const int pos = qa + (col >> p.g_shift), hq = it.h * G + (col & (G - 1));
+      return pos < it.q_end ? -kLog2e * p.lse[(long long)(it.q_row0 + pos - it.q_start) * p.g.hq + hq] : -INFINITY;
+    };
+    static_assert(kRCols == 128, "four lse values per lane");
+    float nl0 = 0.f, nl1 = 0.f, nl2 = 0.f, nl3 = 0.f;
+    if (it.nt > 0) {
+      nl0 = neg_lse(0, 0);
+      nl1 = neg_lse(0, 1);
+      nl2 = neg_lse(0, 2);
+      nl3 = neg_lse(0, 3);
+    }
     for (int t = 0; t < it.nt; ++t, ++qc) {
       const int s = qc % kRStages;
       const uint32_t u = (uint32_t)(qc / kRStages);
+      const int qa = it.k_lo + (it.t0 + t) * p.tile_pos;
       if (!(ok = warp_wait(&bar->q_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
       if (!(ok = warp_wait(&bar->l_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
-      const int qa = it.k_lo + (it.t0 + t) * p.tile_pos;
       float *ls = lse_s + s * kRCols;
-      for (int col = lane; col < kRCols; col += 32) {
-        const int pos = qa + (col >> p.g_shift), hq = it.h * G + (col & (G - 1));
-        ls[col] = pos < it.q_end ? p.lse[(long long)(it.q_row0 + pos - it.q_start) * p.g.hq + hq] * kLog2e
-                                 : INFINITY;
-      }
+      ls[lane] = nl0;
+      ls[lane + 32] = nl1;
+      ls[lane + 64] = nl2;
+      ls[lane + 96] = nl3;
       __syncwarp();
+      if (t + 1 < it.nt) {  // in flight while the next stage frees up
+        nl0 = neg_lse(t + 1, 0);
+        nl1 = neg_lse(t + 1, 1);
+        nl2 = neg_lse(t + 1, 2);
+        nl3 = neg_lse(t + 1, 3);
+      }
       if (lane == 0) {
         mbar_arrive(&bar->l_full[s]);
         mbar_expect_tx(&bar->q_full[s], S::kTileBytes);
@@ -162,7 +202,7 @@ __device__ __forceinline__ void router_producer(const CUtensorMap &qmap, const C
     ++i;
   }
   // drain: no copy of this CTA may still be in flight when it exits
-  if (k_loads > 0) mbar_wait_drain(&bar->k_full, (uint32_t)(k_loads - 1) & 1);
+  for (int k = k_loads - 1; k >= 0 && k >= k_loads - 2; --k) mbar_wait_drain(&bar->k_full[k & 1], (uint32_t)(k >> 1) & 1);
   for (int k = qc - 1; k >= 0 && k >= qc - kRStages; --k)
     mbar_wait_drain(&bar->q_full[k % kRStages], (uint32_t)(k / kRStages) & 1);
 }
@@ -186,7 +226,9 @@ __device__ __forceinline__ void router_mma(const RouterLaunch &p, RBars *bar, co
     mbar_arrive(&bar->sched_empty[slot]);
     if (idx < 0) break;
     const int nt = items[idx].w & 0xFFFFF;
-    if (!(ok = mbar_wait(&bar->k_full, i & 1, abort_flag, state))) break;
+    const int kb = i & 1;
+    if (!(ok = mbar_wait(&bar->k_full[kb], (i >> 1) & 1, abort_flag, state))) break;
+    const uint32_t ka = k_lo + kb * (S::kTileBytes >> 4);
     for (int t = 0; t < nt; ++t, ++qc) {
       const int s = qc % kRStages, buf = qc & 1;
       if (!(ok = mbar_wait(&bar->q_full[s], (uint32_t)(qc / kRStages) & 1, abort_flag, state))) break;
@@ -195,13 +237,13 @@ __device__ __forceinline__ void router_mma(const RouterLaunch &p, RBars *bar, co
       const uint32_t qb = q_lo + s * (S::kTileBytes >> 4);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss(tmem + buf * kRCols, desc(k_lo + (kk >> 2) * (kRKeys * 128 >> 4) + (kk & 3) * 2),
+        umma_ss(tmem + buf * kRCols, desc(ka + (kk >> 2) * (kRKeys * 128 >> 4) + (kk & 3) * 2),
                 desc(qb + (kk >> 2) * (kRCols * 128 >> 4) + (kk & 3) * 2), kIdesc, kk > 0 ? 1u : 0u);
       umma_commit(&bar->s_full[buf]);
       umma_commit(&bar->q_empty[s]);
     }
     if (!ok) break;
-    umma_commit(&bar->k_empty);
+    umma_commit(&bar->k_empty[kb]);
     ++i;
   }
   // every MMA issued by this thread must finish before TMEM is released
@@ -210,12 +252,16 @@ __device__ __forceinline__ void router_mma(const RouterLaunch &p, RBars *bar, co
 }
 
 // ---------------------------------------------------------------------------- reducing warps
+// Warps 4 and up: warp w reads TMEM lane quadrant w mod 4 (32 keys, one per thread) and
+// column group (w - 4) / 4 (kRGroupCols of the 128 query columns of each tile).
 __device__ __forceinline__ void router_reduce(const RouterLaunch &p, RBars *bar, const RouterSeq *seqs,
                                               const int4 *items, const float *lse_s, uint32_t tmem, int warp,
                                               int lane, int32_t *state, volatile int *abort_flag) {
-  const int q4 = warp & 3;  // TMEM lane quadrant this warp may access
+  constexpr int kHalf = kRGroupCols;
+  const int q4 = warp & 3;
+  const int half = (warp - 4) >> 2;  // column group
   const int row = q4 * 32 + lane;
-  const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
+  const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16) + half * kHalf;
   const float sl2 = p.scale_log2;
   const int W = p.g.window;
   int i = 0, qc = 0;
@@ -235,42 +281,47 @@ __device__ __forceinline__ void router_reduce(const RouterLaunch &p, RBars *bar,
       if (!(ok = warp_wait(&bar->l_full[s], (uint32_t)(qc / kRStages) & 1, abort_flag, state))) break;
       if (!(ok = warp_wait(&bar->s_full[buf], (uint32_t)(qc >> 1) & 1, abort_flag, state))) break;
       tc_fence_after();
+      uint32_t r[kHalf];
+#pragma unroll
+      for (int j = 0; j < kHalf / 32; ++j)
+        tmem_ld32(t_lane + buf * kRCols + 32 * j, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * j]));
       const int qa = it.k_lo + (it.t0 + t) * p.tile_pos, q_last = qa + p.tile_pos - 1;
       // every key of the tile sees every query of the tile, and every column is a query
       const bool full = qa >= k0 + kRKeys - 1 && q_last < it.q_end && (it.global || q_last - k0 < W);
-      const float *ls = lse_s + s * kRCols;
-      float tile = 0.f;
-#pragma unroll 1
-      for (int cb = 0; cb < kRCols / 32; ++cb) {
-        uint32_t r[32];
-        tmem_ld32(t_lane + buf * kRCols + cb * 32, r);
-        tmem_ld_wait();
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        if (full) {
+      const float4 *nl = reinterpret_cast<const float4 *>(lse_s + s * kRCols + half * kHalf);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      tmem_ld_wait();
+      if (full) {
+        // (moving a quarter of these exponentials to the FMA pipe with exp2_fma2 measured
+        // 2 % slower: the loop is bound by issue and latency, not by the MUFU)
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            a0 += fast_exp2(fmaf(__uint_as_float(r[c + 0]), sl2, -ls[cb * 32 + c + 0]));
-            a1 += fast_exp2(fmaf(__uint_as_float(r[c + 1]), sl2, -ls[cb * 32 + c + 1]));
-            a2 += fast_exp2(fmaf(__uint_as_float(r[c + 2]), sl2, -ls[cb * 32 + c + 2]));
-            a3 += fast_exp2(fmaf(__uint_as_float(r[c + 3]), sl2, -ls[cb * 32 + c + 3]));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int col = cb * 32 + c;
-            const int qpos = qa + (col >> p.g_shift);
-            const bool vis = kp <= qpos && (it.global || qpos - kp < W);
-            const float e = fast_exp2(fmaf(__uint_as_float(r[c]), sl2, -ls[col]));
-            const float v = vis ? e : 0.f;
-            if ((c & 3) == 0) a0 += v;
-            else if ((c & 3) == 1) a1 += v;
-            else if ((c & 3) == 2) a2 += v;
-            else a3 += v;
-          }
+        for (int c = 0; c < kHalf; c += 4) {
+          const float4 l = nl[c / 4];
+          a0 += fast_exp2(fmaf(__uint_as_float(r[c + 0]), sl2, l.x));
+          a1 += fast_exp2(fmaf(__uint_as_float(r[c + 1]), sl2, l.y));
+          a2 += fast_exp2(fmaf(__uint_as_float(r[c + 2]), sl2, l.z));
+          a3 += fast_exp2(fmaf(__uint_as_float(r[c + 3]), sl2, l.w));
         }
-        tile += (a0 + a1) + (a2 + a3);
+      } else {
+        // key kp sees query position qpos iff kp <= qpos (and qpos - kp < W for a local head);
+        // column c of this half holds position qa + ((col0 + c) >> g_shift), which never
+        // decreases with c, so the visible columns are one range [c_lo, c_hi]
+        const int col0 = half * kHalf;
+        const int c_lo = max(kp - qa, 0) * (1 << p.g_shift) - col0;
+        const int c_hi = it.global ? kHalf : min(kp + W - qa, p.tile_pos) * (1 << p.g_shift) - 1 - col0;
+        auto w = [&](int c, float l) -> float {
+          return (c >= c_lo && c <= c_hi) ? fast_exp2(fmaf(__uint_as_float(r[c]), sl2, l)) : 0.f;
+        };
+#pragma unroll
+        for (int c = 0; c < kHalf; c += 4) {
+          const float4 l = nl[c / 4];
+          a0 += w(c + 0, l.x);
+          a1 += w(c + 1, l.y);
+          a2 += w(c + 2, l.z);
+          a3 += w(c + 3, l.w);
+        }
       }
-      acc += tile;
+      acc += (a0 + a1) + (a2 + a3);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -280,7 +331,8 @@ __device__ __forceinline__ void router_reduce(const RouterLaunch &p, RBars *bar,
     }
     if (!ok) break;
     if (kp >= it.q_start && kp < it.q_end)
-      p.part[((long long)it.chunk * p.g.hkv + it.h) * p.n_tokens + it.q_row0 + (kp - it.q_start)] = acc;
+      p.part[(((long long)it.chunk * kRouterColGroups + half) * p.g.hkv + it.h) * p.n_tokens + it.q_row0 +
+             (kp - it.q_start)] = acc;
     ++i;
   }
 }
@@ -306,22 +358,24 @@ __global__ void __launch_bounds__(kRThreads, 1)
   volatile int *abort_flag = &bar->abort_flag;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar->k_full, 1);
-    mbar_init(&bar->k_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar->k_full[b], 1);
+      mbar_init(&bar->k_empty[b], 1);
+    }
     for (int s = 0; s < kRStages; ++s) {
       mbar_init(&bar->q_full[s], 1);
       mbar_init(&bar->q_empty[s], 1);
       mbar_init(&bar->l_full[s], 1);
-      mbar_init(&bar->l_empty[s], 4);
+      mbar_init(&bar->l_empty[s], kRReducers);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar->s_full[b], 1);
-      mbar_init(&bar->s_empty[b], 4);
+      mbar_init(&bar->s_empty[b], kRReducers);
     }
     mbar_init(&bar->mma_done, 1);
     for (int s = 0; s < 4; ++s) {
       mbar_init(&bar->sched_full[s], 1);
-      mbar_init(&bar->sched_empty[s], 5);  // MMA thread + lane 0 of each reducing warp
+      mbar_init(&bar->sched_empty[s], 1 + kRReducers);  // MMA thread + lane 0 of each reducing warp
     }
     bar->abort_flag = 0;
     fence_mbar_init();
@@ -332,12 +386,16 @@ __global__ void __launch_bounds__(kRThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
-  if (warp == 0) {
-    router_producer<D>(qmap, kmap, p, bar, seqs, items, k_s, q_s, lse_s, sched_next, lane, G, state, abort_flag);
-  } else if (warp == 1) {
-    if (lane == 0) router_mma<D>(p, bar, items, k_s, q_s, tmem, state, abort_flag);
-  } else {
+  if (warp >= 4) {
+    if constexpr (kRSplitRegs) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRRegsHigh));
     router_reduce(p, bar, seqs, items, lse_s, tmem, warp, lane, state, abort_flag);
+  } else {
+    if constexpr (kRSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRRegsLow));
+    if (warp == 0) {
+      router_producer<D>(qmap, kmap, p, bar, seqs, items, k_s, q_s, lse_s, sched_next, lane, G, state, abort_flag);
+    } else if (warp == 1 && lane == 0) {
+      router_mma<D>(p, bar, items, k_s, q_s, tmem, state, abort_flag);
+    }
   }
 
   tc_fence_before();
@@ -380,47 +438,87 @@ __device__ __forceinline__ uint32_t block_scan_excl(uint32_t v, uint32_t *warp_t
   return r;
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float *__restrict__ part, int chunks, int hkv,
-                                                            int n_tokens, const int4 *__restrict__ meta,
-                                                            float *__restrict__ scores, int32_t *__restrict__ rows_out) {
+__global__ void __launch_bounds__(64) score_sum_kernel(const float *__restrict__ part, int slots, int hkv,
+                                                      int n_tokens, float *__restrict__ scores) {
+  const int t = blockIdx.x * 64 + threadIdx.x;
+  if (t >= n_tokens) return;
+  const int n = slots * hkv;  // partial j = (slot, head) at part[j * n_tokens + t]
+  float s = 0.f;
+  int j = 0;
+  for (; j + 8 <= n; j += 8) {  // eight loads in flight, added in order
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = part[(long long)(j + e) * n_tokens + t];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s += v[e];
+  }
+  for (; j < n; ++j) s += part[(long long)j * n_tokens + t];
+  scores[t] = s;
+}
+
+// cache_cap: scores a CTA may keep in dynamic shared memory (a sequence with more tokens
+// reads them from global memory in every pass).
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const int4 *__restrict__ meta,
+                                                            const float *__restrict__ scores_g,
+                                                            int32_t *__restrict__ rows_out, int cache_cap) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_tot[33];
   __shared__ uint32_t sel[2];
+  extern __shared__ float cache[];
   const int4 m = meta[blockIdx.x];
   const int row0 = m.x, n = m.y, k = m.z, out0 = m.w;
   const int tid = threadIdx.x;
-  // scores: the partials of every chunk and KV head, added in that fixed order
-  for (int t = tid; t < n; t += kTopkThreads) {
-    float s = 0.f;
-    for (int c = 0; c < chunks; ++c)
-      for (int h = 0; h < hkv; ++h) s += part[((long long)c * hkv + h) * n_tokens + row0 + t];
-    scores[row0 + t] = s;
-  }
-  __syncthreads();
   if (k <= 0) return;
+  const float *scores = scores_g + row0;
+  if (n <= cache_cap) {
+    for (int t = tid; t < n; t += kTopkThreads) cache[t] = scores[t];
+    __syncthreads();
+    scores = cache;
+  }
   if (k >= n) {
     for (int t = tid; t < n; t += kTopkThreads) rows_out[out0 + t] = row0 + t;
     return;
   }
   // radix select of the k-th largest bit pattern, 8 bits per pass from the top
+  const int lane = tid & 31;
   uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
   for (int shift = 24; shift >= 0; shift -= 8) {
     if (tid < 256) hist[tid] = 0;
     __syncthreads();
-    for (int t = tid; t < n; t += kTopkThreads) {
-      const uint32_t u = __float_as_uint(scores[row0 + t]);
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    for (int base = 0; base < n; base += kTopkThreads) {  // whole warps take part in the match
+      const int t = base + tid;
+      const uint32_t u = t < n ? __float_as_uint(scores[t]) : 0u;
+      const bool in = t < n && (u & mask) == prefix;
+      const uint32_t digit = in ? (u >> shift) & 255u : 256u;
+      // lanes with the same digit add once, through their lowest lane
+      const uint32_t same = __match_any_sync(0xffffffffu, digit);
+      if (in && lane == __ffs(same) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(same));
     }
     __syncthreads();
-    if (tid == 0) {
-      uint32_t above = 0;
-      int d = 255;
-      for (; d > 0; --d) {
-        if (above + hist[d] >= remaining) break;
-        above += hist[d];
+    if (tid < 32) {
+      // lane l owns digits 255 - 8 l down to 248 - 8 l; a suffix scan over lanes finds the
+      // digit at which the count of larger-or-equal candidates reaches `remaining`
+      uint32_t own = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) own += hist[255 - 8 * lane - j];
+      uint32_t incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
       }
-      sel[0] = prefix | ((uint32_t)d << shift);
-      sel[1] = remaining - above;
+      const uint32_t hit = __ballot_sync(0xffffffffu, incl >= remaining);
+      const int l = __ffs(hit) - 1;  // the candidates always reach `remaining`
+      if (lane == l) {
+        uint32_t above = incl - own;
+        int d = 255 - 8 * l;
+        for (int j = 0; j < 7; ++j, --d) {
+          if (above + hist[d] >= remaining) break;
+          above += hist[d];
+        }
+        sel[0] = prefix | ((uint32_t)d << shift);
+        sel[1] = remaining - above;
+      }
     }
     __syncthreads();
     prefix = sel[0];
@@ -432,7 +530,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float *__restr
   uint32_t gt_before = 0, eq_before = 0;
   for (int base = 0; base < n; base += kTopkThreads) {
     const int t = base + tid;
-    const uint32_t u = t < n ? __float_as_uint(scores[row0 + t]) : 0u;
+    const uint32_t u = t < n ? __float_as_uint(scores[t]) : 0u;
     const uint32_t gt = (t < n && u > thr) ? 1u : 0u, eq = (t < n && u == thr) ? 1u : 0u;
     uint32_t total;
     const uint32_t ex = block_scan_excl(gt | (eq << 16), warp_tot, total);
@@ -468,8 +566,19 @@ cudaError_t launch_router(const RouterLaunch &p, const CUtensorMap &qmap, const 
 }
 
 cudaError_t launch_topk(const float *part, int chunks, int hkv, int n_tokens, const int4 *topk_meta, int nseq,
-                        float *scores, int32_t *rows_out, cudaStream_t st) {
-  topk_kernel<<<nseq, kTopkThreads, 0, st>>>(part, chunks, hkv, n_tokens, topk_meta, scores, rows_out);
+                        int max_len, float *scores, int32_t *rows_out, cudaStream_t st) {
+  score_sum_kernel<<<(n_tokens + 63) / 64, 64, 0, st>>>(part, chunks, hkv, n_tokens, scores);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // keep up to 16 384 scores (64 KiB) of a sequence in shared memory
+  constexpr int kCacheCap = 16384;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if ((e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4 * kCacheCap))) return e;
+    attr_set = true;
+  }
+  const int cap = std::min(max_len, kCacheCap);
+  topk_kernel<<<nseq, kTopkThreads, 4 * cap, st>>>(topk_meta, scores, rows_out, cap);
   return cudaGetLastError();
 }
 

@@ -522,7 +522,7 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
                      4 * (size_t)max_batch * Hq * kMaxSplits;
   const size_t rt = router_meta_bytes(max_batch, H * ((size_t)max_tokens / kRouterKeys + 2 * max_batch) *
                                                      kRouterMaxChunks) +
-                    router_part_bytes(kRouterMaxChunks, (int)H, max_tokens);
+                    router_part_bytes(kRouterColGroups * kRouterMaxChunks, (int)H, max_tokens);
   return align_up(std::max(std::max(app, rt), std::max(pre, dec)), 256);
 }
 
@@ -935,8 +935,10 @@ int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
         }
       }
   }
+  // partial slots: (chunk, group of query columns) -- kRouterColGroups reducing warps share each key
   int chunks = 1;
   for (const int4 &it : items) chunks = std::max(chunks, ((int)((uint32_t)it.w >> 20)) + 1);
+  const int slots = kRouterColGroups * chunks;
   {
     std::vector<size_t> order(items.size());
     for (size_t i = 0; i < order.size(); ++i) order[i] = i;
@@ -951,7 +953,7 @@ int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
   const size_t topk_off = items_off + 16 * items.size();
   const size_t bytes = topk_off + 16 * (size_t)nseq;
   const size_t part_off = router_meta_bytes(nseq, items.size());
-  const size_t need = part_off + router_part_bytes(chunks, H, tq);
+  const size_t need = part_off + router_part_bytes(slots, H, tq);
   if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEGKV_ERR_WORKSPACE;
   const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads;
   CUtensorMap qmap;
@@ -977,7 +979,7 @@ int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = upload(h, ws, bytes, st))) return rc;
   float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + part_off);
-  SEGKV_CUDA(h, "router partials clear", cudaMemsetAsync(part, 0, router_part_bytes(chunks, H, tq), st));
+  SEGKV_CUDA(h, "router partials clear", cudaMemsetAsync(part, 0, router_part_bytes(slots, H, tq), st));
   RouterLaunch p{};
   p.g = geom(h);
   p.layer = layer;
@@ -996,8 +998,8 @@ int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
   p.scale_log2 = scale * 1.4426950408889634f;
   if (p.n_items > 0) SEGKV_CUDA(h, "router launch", launch_router(p, qmap, h->kmap, st));
   SEGKV_CUDA(h, "top-k launch",
-             launch_topk(part, chunks, H, (int)tq, reinterpret_cast<const int4 *>(static_cast<char *>(ws) + topk_off),
-                         nseq, scores, rows_out, st));
+             launch_topk(part, slots, H, (int)tq, reinterpret_cast<const int4 *>(static_cast<char *>(ws) + topk_off),
+                         nseq, *std::max_element(q_len, q_len + nseq), scores, rows_out, st));
   return SEGKV_OK;
 }
 

@@ -44,6 +44,7 @@ DECODE = "decode_64x32k"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_SOURCES = ["head_wise_sparse_b200/csrc/prefill_sm100.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 DECODE_SOURCES = ["head_wise_sparse_b200/csrc/decode.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
+ROUTER_SOURCES = ["head_wise_sparse_b200/csrc/router_sm100.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -415,7 +416,8 @@ def main():
               "ms_per_call": t_rt, "pairs_per_call": pairs, "k": k_top[0],
               "step": "segkv_router_topk: received attention mass of 8192 tokens (32 query heads) + top 2048",
               "roofline": {"bound": "alu", "achieved": pairs / (t_rt * 1e-3) / 1e9, "peak": mufu_peak,
-                           "unit": "Gexp/s", "frac": pairs / (t_rt * 1e-3) / 1e9 / mufu_peak, "traffic": None,
+                           "unit": "Gexp/s", "frac": pairs / (t_rt * 1e-3) / 1e9 / mufu_peak,
+                           "traffic": profiled_traffic("router_mistral7b_L8192.md", ROUTER_SOURCES),
                            "peak_source": f"MUFU ex2: 16 per clock per SM x {sms} SMs x {max_mhz:.0f} MHz",
                            "kernel": "router_kernel<128> + score_sum_kernel + topk_kernel (events around segkv_router_topk)"},
               "gpu_launches": 3 * len(evt)}

@@ -141,3 +141,28 @@ def test_plan_matches_oracle_on_random_varlen_batches(seed):
     got, tile_pos, key_tile = h.plan_prefill(0, qs, ql)
     want = orc.lpt_items(qs, ql, cls, W, tile_pos, key_tile)
     assert np.array_equal(got, want)
+
+
+def test_decode_step_validation_happens_before_any_enqueue():
+    h = handle(max_seq_len=64)
+    big = 1 << 20
+    # bad pointers (null K/V or query), bad layer, duplicate ids, negative splits
+    assert h.decode_step(0, [0], 0, FAKE, FAKE, 0.0, 0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.decode_step(0, [0], FAKE, FAKE, 0, 0.0, 0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.decode_step(1, [0], FAKE, FAKE, FAKE, 0.0, 0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.decode_step(0, [2, 2], FAKE, FAKE, FAKE, 0.0, 0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.decode_step(0, [0], FAKE, FAKE, FAKE, 0.0, -1, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.decode_step(0, [0], FAKE + 8, FAKE, FAKE, 0.0, 0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.seq_len(0, 0) == 0 and h.pages_used == 0
+
+
+def test_router_validation_happens_before_any_enqueue():
+    h = handle()
+    big = 1 << 20
+    # queries beyond the sequence (length 0), k above q_len, negative k, misaligned lse
+    assert h.router_topk(0, [0], [0], [4], FAKE, FAKE, 0.0, [1], FAKE, FAKE, FAKE, big, stream=0) == 1
+    assert h.router_topk(0, [0], [0], [0], FAKE, FAKE, 0.0, [1], FAKE, FAKE, FAKE, big, stream=0) == 1
+    assert h.router_topk(0, [0], [0], [0], FAKE, FAKE, 0.0, [-1], FAKE, FAKE, FAKE, big, stream=0) == 1
+    assert h.router_topk(0, [0, 0], [0, 0], [0, 0], FAKE, FAKE, 0.0, [0, 0], FAKE, FAKE, FAKE, big, stream=0) == 1
+    # an empty call (no query tokens) is a no-op
+    assert h.router_topk(0, [0], [0], [0], FAKE, FAKE, 0.0, [0], FAKE, FAKE, FAKE, big, stream=0) == 0

@@ -41,6 +41,7 @@ from head_wise_sparse_b200 import workloads as wl  # noqa: E402
 METRIC = "prefill TFLOP/s over visible (q,k) pairs (% BF16 peak); decode KV GB/s (% HBM)"
 PREFILL = "mistral7b_prefill_L8192"
 DECODE = "decode_64x32k"
+CHUNKED = "mha_chunked_prefill_128k"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_SOURCES = ["head_wise_sparse_b200/csrc/prefill_sm100.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 DECODE_SOURCES = ["head_wise_sparse_b200/csrc/decode.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
@@ -450,6 +451,7 @@ def main():
     line["relocate"] = relocate
     line["router"] = router
     line["fork"] = bench_fork(args, torch, dev, stream, max_over_ranks, world, pk)
+    line["two_source"] = bench_two_source(args, torch, dev, stream, max_over_ranks, world, pk)
     if decode is not None:
         line["decode"] = decode
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -460,6 +462,75 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def bench_two_source(args, torch, dev, stream, max_over_ranks, world, pk):
+    """Chunked prefill of the 128K-context MHA workload (4096 queries at 126976, W 4096, P 64,
+    4 global + 28 local KV heads): segkv_prefill_attn_2src before the chunk is appended, with
+    local rings of ceil((W - 1) / P) + 1 = 65 pages, against segkv_prefill_attn after the
+    append, which needs 129.  Same keys, same FLOPs; the rings hold half the pages."""
+    from head_wise_sparse_b200.segkv import SegKV
+
+    w = wl.CONFIGS[CHUNKED]
+    s = w.seqs[0]
+    ctx, C = s.context, s.new
+    r_two = -(-(w.window - 1) // w.page) + 1
+    handles = {}
+    for name, ring in (("one", w.ring_pages), ("two", r_two)):
+        handles[name] = SegKV(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=w.page,
+                              window=w.window, head_class=w.class_array(), num_pages=w.num_pages,
+                              free_list=w.free_list(), max_seqs=1, max_seq_len=w.max_seq_len, ring_pages=ring,
+                              max_chunk=C, ws_batch=1, ws_tokens=C, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(12)
+    for lo in range(0, ctx, 4096):
+        n = min(4096, ctx - lo)
+        k = (torch.randn((n, w.hkv, w.d), generator=gen, device=dev) / np.sqrt(w.d)).to(torch.bfloat16)
+        v = torch.randn((n, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+        for kv in handles.values():
+            kv.append(0, [0], [lo], [n], k, v)
+        del k, v
+    kc = (torch.randn((C, w.hkv, w.d), generator=gen, device=dev) / np.sqrt(w.d)).to(torch.bfloat16)
+    vc = torch.randn((C, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn((C, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((C, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((C, w.hq), dtype=torch.float32, device=dev)
+    handles["one"].append(0, [0], [ctx], [C], kc, vc)  # the one-source call needs the chunk stored first
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    calls = {"one": lambda: handles["one"].prefill(0, [0], [ctx], [C], q, out=out, lse=lse),
+             "two": lambda: handles["two"].prefill_2src(0, [0], [ctx], [C], q, kc, vc, out=out, lse=lse)}
+    ms = {}
+    for name, call in calls.items():
+        for _ in range(args.warmup):
+            call()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(args.steps, 20))]
+        for e in ev:
+            flush.fill_(3)
+            e[0].record(stream)
+            call()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        ms[name] = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev))
+    handles["two"].append(0, [0], [ctx], [C], kc, vc)
+    torch.cuda.synchronize()
+    for kv in handles.values():
+        if kv.device_status() != 0:
+            raise RuntimeError("device error word set during the two-source benchmark")
+    flops = 4.0 * w.d * visible_pairs(w)
+    n_local = int(w.hkv - sum(w.classes[0]))
+    page_bytes = 2 * w.page * w.d * 2
+    res = {"workload": CHUNKED, "metric": "two-source chunked prefill TFLOP/s", "unit": "TFLOP/s",
+           "value": world * flops / (ms["two"] * 1e-3) / 1e12, "ms_per_call": ms["two"],
+           "one_source_ms_per_call": ms["one"], "ring_pages": {"two_source": r_two, "one_source": w.ring_pages},
+           "local_ring_bytes_saved_per_sequence": n_local * (w.ring_pages - r_two) * page_bytes,
+           "roofline": {"bound": "tensor", "achieved": flops / (ms["two"] * 1e-3) / 1e12, "peak": pk["bf16_tflops"],
+                        "unit": "TFLOP/s", "frac": flops / (ms["two"] * 1e-3) / 1e12 / pk["bf16_tflops"],
+                        "traffic": None, "kernel": "prefill_kernel<128>, chunk pages from the call's K/V "
+                                                   "(events around segkv_prefill_attn_2src)"},
+           "gpu_launches": 2 * len(ev)}
+    del handles, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def bench_fork(args, torch, dev, stream, max_over_ranks, world, pk):

@@ -77,9 +77,13 @@ struct PrefillLaunch {
   float *lse;
   unsigned long long *visited;
   float scale_log2;
+  int two_src;  // 1: pages of each sequence's query range come from kcmap / vcmap, not the pool
 };
+// kcmap / vcmap: the two-source call's K/V tensors [tokens, hkv, D] (box 64 x 1 x page);
+// unused (any valid map) when two_src == 0.
 cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
-                           const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t st);
+                           const CUtensorMap &vmap, const CUtensorMap &omap, const CUtensorMap &kcmap,
+                           const CUtensorMap &vcmap, cudaStream_t st);
 int prefill_smem_bytes(int head_dim);
 
 struct DecodeLaunch {

@@ -77,6 +77,7 @@ struct Smem {
 
 struct Item {
   int b, h, t, q_first, q_last, lo_min, kt_lo, kt_hi, seq_id, kv_len, q_row, slot;
+  int c_start, c_end, c_row0;  // the sequence's query range and its first packed row
   bool global;
 };
 
@@ -109,6 +110,9 @@ __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const Prefil
   const int pair = 2 * p.tile_pos;
   it.seq_id = s.seq_id;
   it.kv_len = s.kv_len;
+  it.c_start = s.q_start;
+  it.c_end = s.q_start + s.q_len;
+  it.c_row0 = s.q_row0;
   it.q_first = s.q_start + it.t * pair;
   it.q_last = s.q_start + min((it.t + 1) * pair, s.q_len) - 1;
   it.q_row = s.q_row0 + it.t * pair;
@@ -120,9 +124,10 @@ __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const Prefil
 }
 
 // ---------------------------------------------------------------------------- producer warp
-template <int D>
+template <int D, bool TWO>
 __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUtensorMap &kmap,
-                                              const CUtensorMap &vmap, const PrefillLaunch &p, Bars *bar,
+                                              const CUtensorMap &vmap, const CUtensorMap &kcmap,
+                                              const CUtensorMap &vcmap, const PrefillLaunch &p, Bars *bar,
                                               const PrefillSeq *seqs, const int4 *items, uint8_t *q_s, uint8_t *k_s,
                                               uint8_t *v_s, int *sched_next, int lane, int G, int32_t *state,
                                               volatile int *abort_flag) {
@@ -131,8 +136,16 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
     tma_prefetch_desc(&qmap);
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
+    if constexpr (TWO) {
+      tma_prefetch_desc(&kcmap);
+      tma_prefetch_desc(&vcmap);
+    }
   }
   const int P = p.g.page, PPT = kBN / P;
+  // Two-source prefill (TWO, a template parameter so the one-source kernel carries none of
+  // it): a page of the call's own query range comes from the caller's K/V tensors, packed
+  // like q; only the context before the range is read from the pages.  Such a page's lane
+  // holds -1 - (its first row in those tensors) instead of a page id.
   int i = 0, c = 0;
   bool ok = true, q_loaded = false;
   // next item index, fetched one item ahead so its Q rows can be pulled into L2 early
@@ -179,12 +192,14 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
         lp_base = lp_first;
         const int lp = lp_base + lane;
         pid = p.g.num_pages;
-        const bool stored = lp <= last_lp && (it.global || lp >= last_lp - p.g.ring + 1);
+        const bool chunk = TWO && lp * P >= it.c_start && lp * P < it.c_end;
+        const bool stored = !chunk && lp <= last_lp && (it.global || lp >= last_lp - p.g.ring + 1);
         if (stored) {
           const int32_t v = p.g.page_table[row_base + (it.global ? lp : lp % p.g.ring)];
           if (v >= 0 && v < p.g.num_pages) pid = v;
           else if ((long long)lp * P + P - 1 >= it.lo_min && lp * P <= it.q_last) set_error(state, kErrDeviceBounds);
         }
+        if (chunk) pid = -1 - (it.c_row0 + lp * P - it.c_start);
       }
       const int s = c % kStages;
       const uint32_t u = (uint32_t)(c / kStages);
@@ -193,18 +208,26 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
       for (int j = 0; j < PPT; ++j) {
         const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
         if (lane == 0)
-          for (int hh = 0; hh < S::kHalves; ++hh)
-            tma_load_3d(k_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, &kmap, &bar->k_full[s], hh * 64, 0,
-                        phys);
+          for (int hh = 0; hh < S::kHalves; ++hh) {
+            uint8_t *dst = k_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128;
+            if (TWO && phys < 0)
+              tma_load_3d(dst, &kcmap, &bar->k_full[s], hh * 64, it.h, -1 - phys);
+            else
+              tma_load_3d(dst, &kmap, &bar->k_full[s], hh * 64, 0, phys);
+          }
       }
       if (!(ok = warp_wait(&bar->v_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
       if (lane == 0) mbar_expect_tx(&bar->v_full[s], S::kTileBytes);
       for (int j = 0; j < PPT; ++j) {
         const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
         if (lane == 0)
-          for (int hh = 0; hh < S::kHalves; ++hh)
-            tma_load_3d(v_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, &vmap, &bar->v_full[s], hh * 64, 0,
-                        phys);
+          for (int hh = 0; hh < S::kHalves; ++hh) {
+            uint8_t *dst = v_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128;
+            if (TWO && phys < 0)
+              tma_load_3d(dst, &vcmap, &bar->v_full[s], hh * 64, it.h, -1 - phys);
+            else
+              tma_load_3d(dst, &vmap, &bar->v_full[s], hh * 64, 0, phys);
+          }
       }
       ++c;
     }
@@ -497,10 +520,11 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
   if ((threadIdx.x & 127) == 0) bulk_wait_all();  // no store of this warpgroup outlives the CTA
 }
 
-template <int D>
+template <int D, bool TWO>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
+                   const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
                    const PrefillLaunch p) {
   using S = Smem<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -557,7 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
-      producer_role<D>(qmap, kmap, vmap, p, bar, seqs, items, q_s, k_s, v_s, sched_next, lane, G, state, abort_flag);
+      producer_role<D, TWO>(qmap, kmap, vmap, kcmap, vcmap, p, bar, seqs, items, q_s, k_s, v_s, sched_next, lane, G, state,
+                       abort_flag);
     } else if (warp == 1 && lane == 0) {
       mma_role<D>(p, bar, seqs, items, q_s, k_s, v_s, tmem, state, abort_flag);
     }
@@ -615,29 +640,30 @@ __global__ void __launch_bounds__(kTileRows) prefill_combine_kernel(const Prefil
 
 int prefill_smem_bytes(int head_dim) { return head_dim == 64 ? Smem<64>::kBytes : Smem<128>::kBytes; }
 
-cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
-                           const CUtensorMap &vmap, const CUtensorMap &omap, cudaStream_t st) {
-  static bool attr_set[2] = {false, false};
-  const int smem = prefill_smem_bytes(p.g.head_dim);
+template <int D, bool TWO>
+static cudaError_t launch_prefill_d(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                                   const CUtensorMap &vmap, const CUtensorMap &omap, const CUtensorMap &kcmap,
+                                   const CUtensorMap &vcmap, cudaStream_t st) {
+  static bool attr_set = false;
+  const int smem = prefill_smem_bytes(D);
   cudaError_t e;
-  if (p.g.head_dim == 64) {
-    if (!attr_set[0]) {
-      if ((e = cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
-        return e;
-      attr_set[0] = true;
-    }
-    prefill_kernel<64><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, p);
-    if (p.n_groups > 0) prefill_combine_kernel<64><<<2 * p.n_groups, kTileRows, 0, st>>>(p);
-  } else {
-    if (!attr_set[1]) {
-      if ((e = cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
-        return e;
-      attr_set[1] = true;
-    }
-    prefill_kernel<128><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, p);
-    if (p.n_groups > 0) prefill_combine_kernel<128><<<2 * p.n_groups, kTileRows, 0, st>>>(p);
+  if (!attr_set) {
+    if ((e = cudaFuncSetAttribute(prefill_kernel<D, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+    attr_set = true;
   }
+  prefill_kernel<D, TWO><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, kcmap, vcmap, p);
+  if (p.n_groups > 0) prefill_combine_kernel<D><<<2 * p.n_groups, kTileRows, 0, st>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                           const CUtensorMap &vmap, const CUtensorMap &omap, const CUtensorMap &kcmap,
+                           const CUtensorMap &vcmap, cudaStream_t st) {
+  if (p.g.head_dim == 64)
+    return p.two_src ? launch_prefill_d<64, true>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st)
+                     : launch_prefill_d<64, false>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st);
+  return p.two_src ? launch_prefill_d<128, true>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st)
+                   : launch_prefill_d<128, false>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st);
 }
 
 }  // namespace skv

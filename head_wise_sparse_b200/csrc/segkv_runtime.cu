@@ -724,24 +724,36 @@ int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_s
   return SEGKV_OK;
 }
 
-int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
-                       const int32_t *q_len, const void *q, float softmax_scale, void *out, float *lse,
-                       uint64_t *visited, void *ws, size_t ws_bytes, void *stream) {
+// Prefill, one-source (k_chunk == NULL: every key from the pages) or two-source (the keys of
+// each sequence's query range from k_chunk / v_chunk, not yet appended).
+static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                        const int32_t *q_len, const void *q, const void *k_chunk, const void *v_chunk,
+                        float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws, size_t ws_bytes,
+                        void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   int rc = check_seqs(h, layer, nseq, seq_ids);
   if (rc) return rc;
   if (!q_start_pos || !q_len) return SEGKV_ERR_INVALID_ARG;
-  const bool has_local = layer_has_local(h, layer);
+  const bool has_local = layer_has_local(h, layer), two = k_chunk != nullptr;
   long long tq = 0;
   for (int b = 0; b < nseq; ++b) {
     const int len = h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]];
-    if (q_len[b] < 0 || q_start_pos[b] < 0 || (long long)q_start_pos[b] + q_len[b] > len) return SEGKV_ERR_INVALID_ARG;
+    if (q_len[b] < 0 || q_start_pos[b] < 0) return SEGKV_ERR_INVALID_ARG;
+    if (two) {
+      // the range starts where the stored sequence ends, on a page boundary
+      if (q_start_pos[b] != len || q_start_pos[b] % h->cfg.page_size != 0 ||
+          (long long)len + q_len[b] > h->cfg.max_seq_len)
+        return SEGKV_ERR_INVALID_ARG;
+    } else if ((long long)q_start_pos[b] + q_len[b] > len) {
+      return SEGKV_ERR_INVALID_ARG;
+    }
     if (q_len[b] > 0 && has_local && !ring_covers(h, len, q_start_pos[b])) return SEGKV_ERR_RING_TOO_SMALL;
     tq += q_len[b];
   }
   if (tq == 0) return SEGKV_OK;
   if (tq > (1LL << 30)) return SEGKV_ERR_UNSUPPORTED;
   if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4)) return SEGKV_ERR_INVALID_ARG;
+  if (two && (!v_chunk || !aligned(k_chunk, 16) || !aligned(v_chunk, 16))) return SEGKV_ERR_INVALID_ARG;
   if ((rc = ensure_device_state(h))) return rc;
   std::vector<PlanItem> items;
   plan_prefill_items(h, layer, nseq, q_start_pos, q_len, items);
@@ -777,12 +789,20 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
     gr[i] = make_int4(g.b, (int)make_item_w1(h->cls[layer * H + g.h] != 0, g.h, g.t), g.first_slot, g.n);
   }
   CUtensorMap qmap, omap;  // query in, output out: the same [tokens, Hq, D] geometry and tile box
-  const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads;
+  const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads, Hkv = h->cfg.num_kv_heads;
   if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
                 kPrefillTileRows / h->G) ||
       !make_map(&omap, out, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
                 kPrefillTileRows / h->G)) {
     h->last_error = "query/output tensor map encode failed";
+    return SEGKV_ERR_CUDA;
+  }
+  CUtensorMap kcmap = h->kmap, vcmap = h->vmap;  // two-source: the call's K/V, one page-sized box per head
+  if (two && (!make_map(&kcmap, k_chunk, D, Hkv, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hkv * D * 2, 1,
+                        h->cfg.page_size) ||
+              !make_map(&vcmap, v_chunk, D, Hkv, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hkv * D * 2, 1,
+                        h->cfg.page_size))) {
+    h->last_error = "chunk K/V tensor map encode failed";
     return SEGKV_ERR_CUDA;
   }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -806,8 +826,25 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
   p.visited = reinterpret_cast<unsigned long long *>(visited);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
-  SEGKV_CUDA(h, "prefill launch", launch_prefill(p, qmap, h->kmap, h->vmap, omap, st));
+  p.two_src = two ? 1 : 0;
+  SEGKV_CUDA(h, "prefill launch", launch_prefill(p, qmap, h->kmap, h->vmap, omap, kcmap, vcmap, st));
   return SEGKV_OK;
+}
+
+int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                       const int32_t *q_len, const void *q, float softmax_scale, void *out, float *lse,
+                       uint64_t *visited, void *ws, size_t ws_bytes, void *stream) {
+  return prefill_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, nullptr, nullptr, softmax_scale, out, lse,
+                      visited, ws, ws_bytes, stream);
+}
+
+int segkv_prefill_attn_2src(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                            const int32_t *q_len, const void *q, const void *k_chunk, const void *v_chunk,
+                            float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws,
+                            size_t ws_bytes, void *stream) {
+  if (!k_chunk) return SEGKV_ERR_INVALID_ARG;
+  return prefill_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, k_chunk, v_chunk, softmax_scale, out, lse,
+                      visited, ws, ws_bytes, stream);
 }
 
 int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,

@@ -26,7 +26,7 @@ EXPORTS = [
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
     "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
     "segkv_decode_attn_noalloc", "segkv_relocate_q", "segkv_fork", "segkv_decode_step",
-    "segkv_router_topk",
+    "segkv_router_topk", "segkv_prefill_attn_2src",
 ]
 
 
@@ -76,6 +76,7 @@ def lib():
         L.segkv_decode_attn_noalloc.argtypes = [P, I, I, P, P, P, F, I, P, P, P, P]
         L.segkv_relocate_q.argtypes = [P, I, I, P, P, P, F, I, P]
         L.segkv_fork.argtypes = [P, I, I, P]
+        L.segkv_prefill_attn_2src.argtypes = [P, I, I, P, P, P, P, P, P, F, P, P, P, P, SZ, P]
         L.segkv_router_topk.argtypes = [P, I, I, P, P, P, P, P, F, P, P, P, P, SZ, P]
         L.segkv_decode_step.argtypes = [P, I, I, P, P, P, P, F, I, P, P, P, P, SZ, P]
         L.segkv_device_status.argtypes = [P, P]
@@ -173,6 +174,13 @@ class Handle:
         s, qs, ql = _i32(seq_ids), _i32(q_start), _i32(q_len)
         return lib().segkv_prefill_attn(self.h, layer, len(s), _p(s), _p(qs), _p(ql), _dptr(q), float(scale),
                                         _dptr(out), _dptr(lse), _dptr(visited), _dptr(ws), ws_bytes, _stream(stream))
+
+    def prefill_2src(self, layer, seq_ids, q_start, q_len, q, k_chunk, v_chunk, scale, out, lse, visited, ws,
+                     ws_bytes, stream=None) -> int:
+        s, qs, ql = _i32(seq_ids), _i32(q_start), _i32(q_len)
+        return lib().segkv_prefill_attn_2src(self.h, layer, len(s), _p(s), _p(qs), _p(ql), _dptr(q), _dptr(k_chunk),
+                                             _dptr(v_chunk), float(scale), _dptr(out), _dptr(lse), _dptr(visited),
+                                             _dptr(ws), ws_bytes, _stream(stream))
 
     def decode(self, layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, ws, ws_bytes,
                stream=None) -> int:
@@ -278,6 +286,18 @@ class SegKV:
         lse = lse if lse is not None else t.empty((T, self.hq), dtype=t.float32, device=self.device)
         _check(self.handle.prefill(layer, seq_ids, q_start, q_len, q, scale, out, lse, visited, self.ws,
                                    self.ws_bytes), "segkv_prefill_attn", self.handle.h)
+        return out, lse
+
+    def prefill_2src(self, layer: int, seq_ids, q_start, q_len, q, k_chunk, v_chunk, *, out=None, lse=None,
+                     visited=None, scale: float = 0.0):
+        """segkv_prefill_attn_2src: prefill of a chunk not yet appended; its keys come from
+        k_chunk / v_chunk [sum(q_len), Hkv, D] (append the chunk afterwards)."""
+        t = self.torch
+        T = int(np.sum(q_len))
+        out = out if out is not None else t.empty((T, self.hq, self.d), dtype=t.bfloat16, device=self.device)
+        lse = lse if lse is not None else t.empty((T, self.hq), dtype=t.float32, device=self.device)
+        _check(self.handle.prefill_2src(layer, seq_ids, q_start, q_len, q, k_chunk, v_chunk, scale, out, lse,
+                                        visited, self.ws, self.ws_bytes), "segkv_prefill_attn_2src", self.handle.h)
         return out, lse
 
     def decode(self, layer: int, seq_ids, q_pos, q, *, out=None, lse=None, visited=None, scale: float = 0.0,

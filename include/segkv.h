@@ -164,6 +164,24 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
                        uint64_t *visited, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Two-source prefill: the same attention as segkv_prefill_attn for a chunk that is NOT yet
+ * appended.  The keys of each sequence's query range come from k_chunk / v_chunk (DEVICE
+ * bf16 [sum(q_len), Hkv, D], packed like q); only the context before the range is read from
+ * the pages.  A local head's ring then needs to hold just the W - 1 tokens before the chunk,
+ * R = ceil((W - 1) / P) + 1 pages, whatever the chunk length (zhichai.net news item "What
+ * Happened", item 3: storage holds only the tokens each head needs).  Append the chunk with
+ * segkv_append afterwards; results equal appending first and calling segkv_prefill_attn,
+ * bit for bit.  Requires q_start_pos[b] == segkv_seq_len(h, layer, seq_ids[b]), a multiple
+ * of the page size.
+ * Errors: INVALID_ARG (range not at the sequence's end or not page-aligned, pointers),
+ * RING_TOO_SMALL, WORKSPACE, CUDA.
+ */
+int segkv_prefill_attn_2src(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                            const int32_t *q_len, const void *q, const void *k_chunk, const void *v_chunk,
+                            float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws,
+                            size_t ws_bytes, void *stream);
+
+/*
  * Longest-processing-time-first work list of the prefill call, before any item is cut into
  * key chunks (host only, no GPU).
  * Item = (b, kv head, query tile, cost); a query tile holds tile_pos = 256 / G consecutive

@@ -18,7 +18,7 @@ FAKE = 1 << 40  # a device address the host never dereferences
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(segkv_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(segkv_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -166,3 +166,15 @@ def test_router_validation_happens_before_any_enqueue():
     assert h.router_topk(0, [0, 0], [0, 0], [0, 0], FAKE, FAKE, 0.0, [0, 0], FAKE, FAKE, FAKE, big, stream=0) == 1
     # an empty call (no query tokens) is a no-op
     assert h.router_topk(0, [0], [0], [0], FAKE, FAKE, 0.0, [0], FAKE, FAKE, FAKE, big, stream=0) == 0
+
+
+def test_two_source_prefill_validation_happens_before_any_enqueue():
+    h = handle()
+    big = 1 << 20
+    # the chunk must start at the sequence's end (0) and on a page boundary
+    assert h.prefill_2src(0, [0], [64], [10], FAKE, FAKE, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    # missing chunk tensors, misaligned chunk tensor
+    assert h.prefill_2src(0, [0], [0], [10], FAKE, 0, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.prefill_2src(0, [0], [0], [10], FAKE, FAKE + 4, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    # past max_seq_len
+    assert h.prefill_2src(0, [0], [0], [4097], FAKE, FAKE, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1

@@ -216,3 +216,33 @@ def test_empty_ranges_single_tokens_and_reset(torch_cuda):
     torch.cuda.synchronize()
     assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
     assert kv.device_status() == 0
+
+
+def test_chunked_128k_two_source_full_size(torch_cuda):
+    # The 4096-token chunk at 126 976 attended before it is appended (segkv_prefill_attn_2src),
+    # with every local ring at ceil((W - 1) / P) + 1 = 65 pages instead of the 129 that the
+    # one-source call needs; sampled rows against the oracle, counts against the closed form.
+    torch = torch_cuda
+    w = wl.CONFIGS["mha_chunked_prefill_128k"]
+    small = w.scaled(ring_pages=-(-(w.window - 1) // w.page) + 1)
+    kv = make_kv(small)
+    o = orc.Oracle.for_workload(w)
+    for ids, st, cnt in context_calls(w, 4096):
+        k, v = kv_for_call(w, 0, ids, st, cnt)
+        kv.append(0, ids, st, cnt, to_dev(k), to_dev(v))
+        o.append(0, ids, st, cnt, k, v)
+    ids, st, cnt = step_append(w)
+    k, v = kv_for_call(w, 0, ids, st, cnt)
+    o.append(0, ids, st, cnt, k, v)
+    qids, qs, ql = step_queries(w)
+    assert (qids, qs, ql) == (ids, st, cnt)  # the chunk is the query range
+    q = q_for_call(w, 0, qids, qs, ql)
+    vis = torch.zeros((len(qids), w.hq), dtype=torch.int64, device="cuda")
+    out, lse = kv.prefill_2src(0, qids, qs, ql, to_dev(q), to_dev(k), to_dev(v), visited=vis)
+    kv.append(0, ids, st, cnt, to_dev(k), to_dev(v))
+    torch.cuda.synchronize()
+    assert kv.device_status() == 0
+    rows = sample_rows(w, ql, 2000, seed=7)
+    ro, rl, _ = o.attention(0, qids, qs, ql, q, rows=rows)
+    compare_rows(w, out, lse, ro, rl, rows)
+    assert np.array_equal(vis.cpu().numpy().astype(np.uint64), closed_form_counts(w, 0, qids, qs, ql))

@@ -21,7 +21,7 @@
 //               4-deep ring, each with the 128 negated lse values of its columns (log2
 //               domain, loaded one tile ahead; -inf marks a column past the sequence's
 //               queries, whose weight is then exactly 0)
-//   warp 1      lane 0 issues the MMAs into two 128-column S buffers in TMEM
+//   warp 1      lane 0 issues the MMAs into four 128-column S buffers in TMEM
 //   warps 2, 3  idle
 //   warps 4..19 four warps per TMEM lane quadrant, each summing 32 of the 128 columns of
 //               its 32 keys (one key per thread); a key's sums over the item go to the
@@ -44,6 +44,7 @@ namespace {
 constexpr int kRKeys = 128;     // keys of a tile (M of the MMA, TMEM lanes)
 constexpr int kRCols = 128;     // query rows of a tile (N of the MMA)
 constexpr int kRStages = 4;     // query-tile ring depth
+constexpr int kRSBufs = 4;      // S buffers in TMEM (4 x 128 columns: all of it)
 constexpr int kRReducers = 4 * kRouterColGroups;  // reducing warps: kRouterColGroups per lane quadrant
 constexpr int kRGroupCols = kRCols / kRouterColGroups;
 constexpr int kRThreads = 128 + 32 * kRReducers;
@@ -70,7 +71,7 @@ struct RSmem {
 struct RBars {
   uint64_t k_full[2], k_empty[2];
   uint64_t q_full[kRStages], q_empty[kRStages], l_full[kRStages], l_empty[kRStages];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[kRSBufs], s_empty[kRSBufs];
   uint64_t mma_done;
   uint64_t sched_full[4], sched_empty[4];
   int sched[4];
@@ -230,9 +231,9 @@ __device__ __forceinline__ void router_mma(const RouterLaunch &p, RBars *bar, co
     if (!(ok = mbar_wait(&bar->k_full[kb], (i >> 1) & 1, abort_flag, state))) break;
     const uint32_t ka = k_lo + kb * (S::kTileBytes >> 4);
     for (int t = 0; t < nt; ++t, ++qc) {
-      const int s = qc % kRStages, buf = qc & 1;
+      const int s = qc % kRStages, buf = qc % kRSBufs;
       if (!(ok = mbar_wait(&bar->q_full[s], (uint32_t)(qc / kRStages) & 1, abort_flag, state))) break;
-      if (!(ok = mbar_wait(&bar->s_empty[buf], ((uint32_t)(qc >> 1) & 1) ^ 1, abort_flag, state))) break;
+      if (!(ok = mbar_wait(&bar->s_empty[buf], ((uint32_t)(qc / kRSBufs) & 1) ^ 1, abort_flag, state))) break;
       tc_fence_after();
       const uint32_t qb = q_lo + s * (S::kTileBytes >> 4);
 #pragma unroll
@@ -277,9 +278,9 @@ __device__ __forceinline__ void router_reduce(const RouterLaunch &p, RBars *bar,
     float acc = 0.f;
     bool ok = true;
     for (int t = 0; t < it.nt; ++t, ++qc) {
-      const int s = qc % kRStages, buf = qc & 1;
+      const int s = qc % kRStages, buf = qc % kRSBufs;
       if (!(ok = warp_wait(&bar->l_full[s], (uint32_t)(qc / kRStages) & 1, abort_flag, state))) break;
-      if (!(ok = warp_wait(&bar->s_full[buf], (uint32_t)(qc >> 1) & 1, abort_flag, state))) break;
+      if (!(ok = warp_wait(&bar->s_full[buf], (uint32_t)(qc / kRSBufs) & 1, abort_flag, state))) break;
       tc_fence_after();
       uint32_t r[kHalf];
 #pragma unroll
@@ -289,7 +290,10 @@ __device__ __forceinline__ void router_reduce(const RouterLaunch &p, RBars *bar,
       // every key of the tile sees every query of the tile, and every column is a query
       const bool full = qa >= k0 + kRKeys - 1 && q_last < it.q_end && (it.global || q_last - k0 < W);
       const float4 *nl = reinterpret_cast<const float4 *>(lse_s + s * kRCols + half * kHalf);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      // pairs of columns through the packed fp32 pipe: one fma.f32x2 forms two exponents, one
+      // add.f32x2 adds two weights, so a column costs two issue slots besides its ex2
+      const float2 sl2v = make_float2(sl2, sl2);
+      float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
       tmem_ld_wait();
       if (full) {
         // (moving a quarter of these exponentials to the FMA pipe with exp2_fma2 measured
@@ -297,31 +301,33 @@ __device__ __forceinline__ void router_reduce(const RouterLaunch &p, RBars *bar,
 #pragma unroll
         for (int c = 0; c < kHalf; c += 4) {
           const float4 l = nl[c / 4];
-          a0 += fast_exp2(fmaf(__uint_as_float(r[c + 0]), sl2, l.x));
-          a1 += fast_exp2(fmaf(__uint_as_float(r[c + 1]), sl2, l.y));
-          a2 += fast_exp2(fmaf(__uint_as_float(r[c + 2]), sl2, l.z));
-          a3 += fast_exp2(fmaf(__uint_as_float(r[c + 3]), sl2, l.w));
+          const float2 x01 = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v,
+                                   make_float2(l.x, l.y));
+          const float2 x23 = ffma2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), sl2v,
+                                   make_float2(l.z, l.w));
+          a01 = fadd2(a01, make_float2(fast_exp2(x01.x), fast_exp2(x01.y)));
+          a23 = fadd2(a23, make_float2(fast_exp2(x23.x), fast_exp2(x23.y)));
         }
       } else {
         // key kp sees query position qpos iff kp <= qpos (and qpos - kp < W for a local head);
-        // column c of this half holds position qa + ((col0 + c) >> g_shift), which never
+        // column c of this group holds position qa + ((col0 + c) >> g_shift), which never
         // decreases with c, so the visible columns are one range [c_lo, c_hi]
         const int col0 = half * kHalf;
         const int c_lo = max(kp - qa, 0) * (1 << p.g_shift) - col0;
         const int c_hi = it.global ? kHalf : min(kp + W - qa, p.tile_pos) * (1 << p.g_shift) - 1 - col0;
-        auto w = [&](int c, float l) -> float {
-          return (c >= c_lo && c <= c_hi) ? fast_exp2(fmaf(__uint_as_float(r[c]), sl2, l)) : 0.f;
-        };
+        auto w = [&](int c, float x) -> float { return (c >= c_lo && c <= c_hi) ? fast_exp2(x) : 0.f; };
 #pragma unroll
         for (int c = 0; c < kHalf; c += 4) {
           const float4 l = nl[c / 4];
-          a0 += w(c + 0, l.x);
-          a1 += w(c + 1, l.y);
-          a2 += w(c + 2, l.z);
-          a3 += w(c + 3, l.w);
+          const float2 x01 = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v,
+                                   make_float2(l.x, l.y));
+          const float2 x23 = ffma2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), sl2v,
+                                   make_float2(l.z, l.w));
+          a01 = fadd2(a01, make_float2(w(c, x01.x), w(c + 1, x01.y)));
+          a23 = fadd2(a23, make_float2(w(c + 2, x23.x), w(c + 3, x23.y)));
         }
       }
-      acc += (a0 + a1) + (a2 + a3);
+      acc += (a01.x + a01.y) + (a23.x + a23.y);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -368,7 +374,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       mbar_init(&bar->l_full[s], 1);
       mbar_init(&bar->l_empty[s], kRReducers);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kRSBufs; ++b) {
       mbar_init(&bar->s_full[b], 1);
       mbar_init(&bar->s_empty[b], kRReducers);
     }
@@ -380,7 +386,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     bar->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(&bar->tmem_base, 2 * kRCols);
+  if (warp == 1) tmem_alloc(&bar->tmem_base, kRSBufs * kRCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -402,7 +408,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * kRCols);
+    tmem_dealloc(tmem, kRSBufs * kRCols);
   }
 }
 

@@ -37,6 +37,24 @@ __host__ __device__ inline uint32_t make_item_w1(bool global, int head, int tile
   return ((uint32_t)global << 31) | ((uint32_t)head << 20) | (uint32_t)tile;
 }
 
+__host__ __device__ inline int max_i(int a, int b) { return a > b ? a : b; }
+
+// Rank of logical page lp among the pages this call allocates for one (sequence, head),
+// in ascending lp (the allocation order), or -1 when lp's slot was allocated before the
+// call.  hb = slots the head held before the call.  A global head's slot is lp, so its new
+// pages are lp >= hb.  A local head fills ring slots 0, 1, ... in order until it holds R, so
+// a slot is new exactly when its index is >= hb; the call touches the last R pages
+// [lp0, lp1], whose slots form a cyclic run starting at lp0 mod R.  (Used when the call
+// copies no shared page: then "allocated" depends only on the sequence's length, also for a
+// fork, which takes its source's length with its page-table rows.)
+__host__ __device__ inline int new_page_rank(int lp, int lp0, int hb, bool global, int R) {
+  if (global) return lp >= hb ? lp - hb : -1;
+  if (lp % R < hb) return -1;
+  const int s0 = lp0 % R, m = lp - lp0;  // new slots among lp0 .. lp-1
+  if (s0 + m <= R) return max_i(0, s0 + m - max_i(s0, hb));
+  return max_i(0, R - max_i(s0, hb)) + max_i(0, s0 + m - R - hb);
+}
+
 struct StorageGeom {  // what every kernel needs to resolve a logical position to a page
   int32_t *page_table;
   const int32_t *free_list;
@@ -78,6 +96,14 @@ struct PrefillLaunch {
   unsigned long long *visited;
   float scale_log2;
   int two_src;  // 1: pages of each sequence's query range come from kcmap / vcmap, not the pool
+  // Fused append (store == 1, with two_src): the item whose query range holds a chunk page's
+  // first position also stores that page from shared memory into the pool (TMA store) and
+  // records it in the page table; a page the call allocates takes free-list entry
+  // cursor0 + pair_off[sequence * hkv + head] + new_page_rank.  Block 0 sets state[0] =
+  // cursor0 + new_pages.
+  int store;
+  const int32_t *pair_off;
+  int cursor0, new_pages;
 };
 // kcmap / vcmap: the two-source call's K/V tensors [tokens, hkv, D] (box 64 x 1 x page);
 // unused (any valid map) when two_src == 0.

@@ -124,7 +124,7 @@ __device__ __forceinline__ Item decode_item(const PrefillLaunch &p, const Prefil
 }
 
 // ---------------------------------------------------------------------------- producer warp
-template <int D, bool TWO>
+template <int D, bool TWO, bool STORE>
 __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUtensorMap &kmap,
                                               const CUtensorMap &vmap, const CUtensorMap &kcmap,
                                               const CUtensorMap &vcmap, const PrefillLaunch &p, Bars *bar,
@@ -146,6 +146,10 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
   // it): a page of the call's own query range comes from the caller's K/V tensors, packed
   // like q; only the context before the range is read from the pages.  Such a page's lane
   // holds -1 - (its first row in those tensors) instead of a page id.
+  // Fused append (STORE): once such a page has landed in shared memory, the item whose query
+  // range holds the page's first position also writes it to its pool page by TMA store, so
+  // every chunk page is stored exactly once; a stage is reloaded only after those stores
+  // have read it.
   int i = 0, c = 0;
   bool ok = true, q_loaded = false;
   // next item index, fetched one item ahead so its Q rows can be pulled into L2 early
@@ -204,6 +208,9 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
       const int s = c % kStages;
       const uint32_t u = (uint32_t)(c / kStages);
       if (!(ok = warp_wait(&bar->k_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
+      if constexpr (STORE) {
+        if (lane == 0) bulk_wait_read_all();  // earlier stores from this stage have read it
+      }
       if (lane == 0) mbar_expect_tx(&bar->k_full[s], S::kTileBytes);
       for (int j = 0; j < PPT; ++j) {
         const int phys = __shfl_sync(0xffffffffu, pid, lp_first + j - lp_base);
@@ -229,6 +236,45 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
               tma_load_3d(dst, &vmap, &bar->v_full[s], hh * 64, 0, phys);
           }
       }
+      if constexpr (STORE) {
+        // lane j: page j of this tile, if this item stores it (its id, else -1)
+        int sp = -1;
+        if (lane < PPT) {
+          const int lp = lp_first + lane, pos = lp * P, R = p.g.ring;
+          const int lp1 = (it.c_end - 1) / P, held = it.c_start / P;
+          if (pos >= it.c_start && pos < it.c_end && pos >= it.q_first && pos <= it.q_last &&
+              (it.global || lp >= lp1 - R + 1)) {
+            const int lp0 = it.global ? held : max(held, lp1 - R + 1);
+            const int rank = new_page_rank(lp, lp0, it.global ? held : min(held, R), it.global, R);
+            const long long slot = row_base + (it.global ? lp : lp % R);
+            const int k = rank >= 0 ? p.cursor0 + p.pair_off[it.b * p.g.hkv + it.h] + rank : -1;
+            const int32_t phys = k >= 0 ? (k < p.g.num_pages ? p.g.free_list[k] : -1) : p.g.page_table[slot];
+            if (phys >= 0 && phys < p.g.num_pages) {
+              if (k >= 0) p.g.page_table[slot] = phys;
+              sp = phys;
+            } else {
+              set_error(state, kErrDeviceBounds);
+            }
+          }
+        }
+        if (__ballot_sync(0xffffffffu, sp >= 0)) {
+          if (!(ok = warp_wait(&bar->k_full[s], u & 1, abort_flag, state))) break;
+          for (int j = 0; j < PPT; ++j) {
+            const int ph = __shfl_sync(0xffffffffu, sp, j);
+            if (lane == 0 && ph >= 0)
+              for (int hh = 0; hh < S::kHalves; ++hh)
+                tma_store_3d(&kmap, k_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, hh * 64, 0, ph);
+          }
+          if (!(ok = warp_wait(&bar->v_full[s], u & 1, abort_flag, state))) break;
+          for (int j = 0; j < PPT; ++j) {
+            const int ph = __shfl_sync(0xffffffffu, sp, j);
+            if (lane == 0 && ph >= 0)
+              for (int hh = 0; hh < S::kHalves; ++hh)
+                tma_store_3d(&vmap, v_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, hh * 64, 0, ph);
+          }
+          if (lane == 0) bulk_commit();
+        }
+      }
       ++c;
     }
     if (!ok) break;
@@ -243,6 +289,9 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
     mbar_wait_drain(&bar->v_full[s], u & 1);
   }
   if (q_loaded) mbar_wait_drain(&bar->q_full, (uint32_t)((ok ? i - 1 : i) & 1));
+  if constexpr (STORE) {
+    if (lane == 0) bulk_wait_all();  // the pool holds every stored page before the CTA exits
+  }
 }
 
 // ---------------------------------------------------------------------------- MMA thread
@@ -520,7 +569,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
   if ((threadIdx.x & 127) == 0) bulk_wait_all();  // no store of this warpgroup outlives the CTA
 }
 
-template <int D, bool TWO>
+template <int D, bool TWO, bool STORE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
@@ -567,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     bar->abort_flag = 0;
     fence_mbar_init();
+    if (STORE && blockIdx.x == 0) state[0] = p.cursor0 + p.new_pages;
   }
   if (warp == 1) tmem_alloc(&bar->tmem_base, 512);
   tc_fence_before();
@@ -581,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
-      producer_role<D, TWO>(qmap, kmap, vmap, kcmap, vcmap, p, bar, seqs, items, q_s, k_s, v_s, sched_next, lane, G, state,
+      producer_role<D, TWO, STORE>(qmap, kmap, vmap, kcmap, vcmap, p, bar, seqs, items, q_s, k_s, v_s, sched_next, lane, G, state,
                        abort_flag);
     } else if (warp == 1 && lane == 0) {
       mma_role<D>(p, bar, seqs, items, q_s, k_s, v_s, tmem, state, abort_flag);
@@ -640,7 +690,7 @@ __global__ void __launch_bounds__(kTileRows) prefill_combine_kernel(const Prefil
 
 int prefill_smem_bytes(int head_dim) { return head_dim == 64 ? Smem<64>::kBytes : Smem<128>::kBytes; }
 
-template <int D, bool TWO>
+template <int D, bool TWO, bool STORE>
 static cudaError_t launch_prefill_d(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
                                    const CUtensorMap &vmap, const CUtensorMap &omap, const CUtensorMap &kcmap,
                                    const CUtensorMap &vcmap, cudaStream_t st) {
@@ -648,22 +698,30 @@ static cudaError_t launch_prefill_d(const PrefillLaunch &p, const CUtensorMap &q
   const int smem = prefill_smem_bytes(D);
   cudaError_t e;
   if (!attr_set) {
-    if ((e = cudaFuncSetAttribute(prefill_kernel<D, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+    if ((e = cudaFuncSetAttribute(prefill_kernel<D, TWO, STORE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem)))
+      return e;
     attr_set = true;
   }
-  prefill_kernel<D, TWO><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, kcmap, vcmap, p);
+  prefill_kernel<D, TWO, STORE><<<p.grid, kThreads, smem, st>>>(qmap, kmap, vmap, omap, kcmap, vcmap, p);
   if (p.n_groups > 0) prefill_combine_kernel<D><<<2 * p.n_groups, kTileRows, 0, st>>>(p);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_prefill_mode(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                                       const CUtensorMap &vmap, const CUtensorMap &omap, const CUtensorMap &kcmap,
+                                       const CUtensorMap &vcmap, cudaStream_t st) {
+  if (!p.two_src) return launch_prefill_d<D, false, false>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st);
+  if (!p.store) return launch_prefill_d<D, true, false>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st);
+  return launch_prefill_d<D, true, true>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st);
 }
 
 cudaError_t launch_prefill(const PrefillLaunch &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
                            const CUtensorMap &vmap, const CUtensorMap &omap, const CUtensorMap &kcmap,
                            const CUtensorMap &vcmap, cudaStream_t st) {
-  if (p.g.head_dim == 64)
-    return p.two_src ? launch_prefill_d<64, true>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st)
-                     : launch_prefill_d<64, false>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st);
-  return p.two_src ? launch_prefill_d<128, true>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st)
-                   : launch_prefill_d<128, false>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st);
+  return p.g.head_dim == 64 ? launch_prefill_mode<64>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st)
+                            : launch_prefill_mode<128>(p, qmap, kmap, vmap, omap, kcmap, vcmap, st);
 }
 
 }  // namespace skv

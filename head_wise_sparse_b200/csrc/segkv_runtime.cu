@@ -511,8 +511,10 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
   const size_t app = align_up(kHeaderBytes + sizeof(AppendSeq) * max_batch + align_up(H, 4) + 4 * (H * max_batch + 1),
                               16) +
                      sizeof(int4) * H * ((size_t)ceil_div(max_tokens, h->cfg.page_size) + 2 * max_batch);
+  // prefill: items, the key-chunk groups and (fused append) one page offset per (sequence, head)
   const size_t pre = prefill_meta_bytes(max_batch, H * ((size_t)ceil_div(max_tokens, tile_pos) + max_batch) +
-                                                      kMaxPartSlots, kMaxPartSlots) +
+                                                      kMaxPartSlots + (H * max_batch + 3) / 4,
+                                        kMaxPartSlots) +
                      prefill_part_bytes((int)D);
   // decode: split counts and (decode step) new page ids per (sequence, head), then the items
   const size_t dec_meta = align_up(kHeaderBytes + sizeof(DecodeSeq) * max_batch + 8 * max_batch * H +
@@ -725,11 +727,12 @@ int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_s
 }
 
 // Prefill, one-source (k_chunk == NULL: every key from the pages) or two-source (the keys of
-// each sequence's query range from k_chunk / v_chunk, not yet appended).
+// each sequence's query range from k_chunk / v_chunk, not yet appended); with `fused`, the
+// kernel also appends those keys (segkv_prefill_append).
 static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
                         const int32_t *q_len, const void *q, const void *k_chunk, const void *v_chunk,
                         float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws, size_t ws_bytes,
-                        void *stream) {
+                        void *stream, bool fused = false) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   int rc = check_seqs(h, layer, nseq, seq_ids);
   if (rc) return rc;
@@ -748,12 +751,50 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
       return SEGKV_ERR_INVALID_ARG;
     }
     if (q_len[b] > 0 && has_local && !ring_covers(h, len, q_start_pos[b])) return SEGKV_ERR_RING_TOO_SMALL;
+    // fused: after the call the ring must still hold every key a query of the call needs
+    // (the one-source rule), so no page the call overwrites in place is read by the call
+    if (fused && q_len[b] > 0 && has_local && !ring_covers(h, len + q_len[b], q_start_pos[b]))
+      return SEGKV_ERR_RING_TOO_SMALL;
     tq += q_len[b];
   }
   if (tq == 0) return SEGKV_OK;
   if (tq > (1LL << 30)) return SEGKV_ERR_UNSUPPORTED;
   if (!q || !out || !lse || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4)) return SEGKV_ERR_INVALID_ARG;
   if (two && (!v_chunk || !aligned(k_chunk, 16) || !aligned(v_chunk, 16))) return SEGKV_ERR_INVALID_ARG;
+  const int H = h->cfg.num_kv_heads, P = h->cfg.page_size, R = h->ring;
+  // fused append, page rule of segkv_append: every empty slot the call touches takes the next
+  // free-list entry (sequence in call order, head ascending, page ascending); pair_off holds
+  // the pages taken by earlier (sequence, head) pairs
+  std::vector<int32_t> pair_off;
+  long long new_pages = 0;
+  auto touched = [&](int b, int k, int &lp0, int &lp1, size_t &row, bool &global) {
+    global = h->cls[layer * H + k] != 0;
+    lp1 = (q_start_pos[b] + q_len[b] - 1) / P;
+    lp0 = q_start_pos[b] / P;
+    if (!global && lp1 - R + 1 > lp0) lp0 = lp1 - R + 1;
+    row = (((size_t)layer * h->cfg.max_seqs + seq_ids[b]) * H + k) * h->max_lp;
+  };
+  if (fused) {
+    if (h->n_shared > 0) {
+      // a page may be shared after a fork: the append's copy on write runs as its own call
+      if ((rc = segkv_append(h, layer, nseq, seq_ids, q_start_pos, q_len, k_chunk, v_chunk, ws, ws_bytes, stream)))
+        return rc;
+      return prefill_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, nullptr, nullptr, softmax_scale, out, lse,
+                          visited, ws, ws_bytes, stream);
+    }
+    pair_off.assign((size_t)nseq * H, 0);
+    for (int b = 0; b < nseq; ++b)
+      for (int k = 0; k < H; ++k) {
+        pair_off[(size_t)b * H + k] = (int32_t)new_pages;
+        if (q_len[b] == 0) continue;
+        int lp0, lp1;
+        size_t row;
+        bool global;
+        touched(b, k, lp0, lp1, row, global);
+        for (int lp = lp0; lp <= lp1; ++lp) new_pages += h->slot_k[row + (global ? lp : lp % R)] < 0;
+      }
+    if (h->pages_used + new_pages > h->cfg.num_pages) return SEGKV_ERR_OUT_OF_PAGES;
+  }
   if ((rc = ensure_device_state(h))) return rc;
   std::vector<PlanItem> items;
   plan_prefill_items(h, layer, nseq, q_start_pos, q_len, items);
@@ -762,8 +803,10 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
   split_long_items(h, layer, q_start_pos, q_len, items, h->num_sms, chunks, groups);
   const int items_off = (int)align_up(kHeaderBytes + sizeof(PrefillSeq) * nseq, 16);
   const int groups_off = items_off + 16 * (int)chunks.size();
-  const size_t bytes = groups_off + 16 * groups.size();
-  const size_t meta = prefill_meta_bytes(nseq, chunks.size(), groups.size());
+  const int pair_off_at = groups_off + 16 * (int)groups.size();
+  const size_t pair_words = align_up(4 * pair_off.size(), 16) / 16;  // in 16-byte units
+  const size_t bytes = pair_off_at + 16 * pair_words;
+  const size_t meta = prefill_meta_bytes(nseq, chunks.size() + pair_words, groups.size());
   const size_t need = meta + prefill_part_bytes(h->cfg.head_dim);
   if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEGKV_ERR_WORKSPACE;
   void *host = nullptr;
@@ -777,7 +820,6 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
     row0 += q_len[b];
   }
   int4 *it = reinterpret_cast<int4 *>(static_cast<char *>(host) + items_off);
-  const int H = h->cfg.num_kv_heads;
   for (size_t i = 0; i < chunks.size(); ++i) {
     const PlanChunk &c = chunks[i];
     it[i] = make_int4(c.b, (int)make_item_w1(h->cls[layer * H + c.h] != 0, c.h, c.t), (c.kt_a << 16) | c.kt_b,
@@ -788,6 +830,7 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
     const SplitGroup &g = groups[i];
     gr[i] = make_int4(g.b, (int)make_item_w1(h->cls[layer * H + g.h] != 0, g.h, g.t), g.first_slot, g.n);
   }
+  if (!pair_off.empty()) std::memcpy(static_cast<char *>(host) + pair_off_at, pair_off.data(), 4 * pair_off.size());
   CUtensorMap qmap, omap;  // query in, output out: the same [tokens, Hq, D] geometry and tile box
   const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads, Hkv = h->cfg.num_kv_heads;
   if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
@@ -827,7 +870,33 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.two_src = two ? 1 : 0;
+  if (fused) {
+    p.store = 1;
+    p.pair_off = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + pair_off_at);
+    p.cursor0 = (int)h->pages_used;
+    p.new_pages = (int)new_pages;
+  }
   SEGKV_CUDA(h, "prefill launch", launch_prefill(p, qmap, h->kmap, h->vmap, omap, kcmap, vcmap, st));
+  if (fused) {  // the host mirror follows the kernel's closed form, in the allocation order
+    int32_t k_new = (int32_t)h->pages_used;
+    for (int b = 0; b < nseq; ++b) {
+      for (int k = 0; k < H && q_len[b] > 0; ++k) {
+        int lp0, lp1;
+        size_t row;
+        bool global;
+        touched(b, k, lp0, lp1, row, global);
+        for (int lp = lp0; lp <= lp1; ++lp) {
+          int32_t &slot = h->slot_k[row + (global ? lp : lp % R)];
+          if (slot < 0) {
+            slot = k_new;
+            h->ref[k_new++] = 1;
+          }
+        }
+      }
+      h->len[(size_t)layer * h->cfg.max_seqs + seq_ids[b]] += q_len[b];
+    }
+    h->pages_used += new_pages;
+  }
   return SEGKV_OK;
 }
 
@@ -836,6 +905,15 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
                        uint64_t *visited, void *ws, size_t ws_bytes, void *stream) {
   return prefill_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, nullptr, nullptr, softmax_scale, out, lse,
                       visited, ws, ws_bytes, stream);
+}
+
+int segkv_prefill_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                         const int32_t *q_len, const void *q, const void *k_new, const void *v_new,
+                         float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws, size_t ws_bytes,
+                         void *stream) {
+  if (!k_new) return SEGKV_ERR_INVALID_ARG;
+  return prefill_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, k_new, v_new, softmax_scale, out, lse,
+                      visited, ws, ws_bytes, stream, true);
 }
 
 int segkv_prefill_attn_2src(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,

@@ -35,21 +35,6 @@ __device__ __forceinline__ void touched_pages(int first, int last, int P, int R,
 }
 
 // ---------------------------------------------------------------------------- append
-// Rank of logical page lp among the pages this call allocates for one (sequence, head),
-// in ascending lp (the allocation order), or -1 when lp's slot was allocated before the
-// call.  hb = slots the head held before the call.  A global head's slot is lp, so its new
-// pages are lp >= hb.  A local head fills ring slots 0, 1, ... in order until it holds R, so
-// a slot is new exactly when its index is >= hb; the call touches the last R pages
-// [lp0, lp1], whose slots form a cyclic run starting at lp0 mod R.  (Used when the call
-// copies no shared page: then "allocated" depends only on the sequence's length, also for a
-// fork, which takes its source's length with its page-table rows.)
-__device__ __forceinline__ int new_page_rank(int lp, int lp0, int hb, bool global, int R) {
-  if (global) return lp >= hb ? lp - hb : -1;
-  if (lp % R < hb) return -1;
-  const int s0 = lp0 % R, m = lp - lp0;  // new slots among lp0 .. lp-1
-  if (s0 + m <= R) return max(0, s0 + m - max(s0, hb));
-  return max(0, R - max(s0, hb)) + max(0, s0 + m - R - hb);
-}
 
 // ---------------------------------------------------------------------------- copy on write
 // One thread per (job, row, 16-byte chunk): job j = (k_new, k_old, rows) copies rows

@@ -26,7 +26,7 @@ EXPORTS = [
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
     "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
     "segkv_decode_attn_noalloc", "segkv_relocate_q", "segkv_fork", "segkv_decode_step",
-    "segkv_router_topk", "segkv_prefill_attn_2src",
+    "segkv_router_topk", "segkv_prefill_attn_2src", "segkv_prefill_append",
 ]
 
 
@@ -77,6 +77,7 @@ def lib():
         L.segkv_relocate_q.argtypes = [P, I, I, P, P, P, F, I, P]
         L.segkv_fork.argtypes = [P, I, I, P]
         L.segkv_prefill_attn_2src.argtypes = [P, I, I, P, P, P, P, P, P, F, P, P, P, P, SZ, P]
+        L.segkv_prefill_append.argtypes = [P, I, I, P, P, P, P, P, P, F, P, P, P, P, SZ, P]
         L.segkv_router_topk.argtypes = [P, I, I, P, P, P, P, P, F, P, P, P, P, SZ, P]
         L.segkv_decode_step.argtypes = [P, I, I, P, P, P, P, F, I, P, P, P, P, SZ, P]
         L.segkv_device_status.argtypes = [P, P]
@@ -181,6 +182,13 @@ class Handle:
         return lib().segkv_prefill_attn_2src(self.h, layer, len(s), _p(s), _p(qs), _p(ql), _dptr(q), _dptr(k_chunk),
                                              _dptr(v_chunk), float(scale), _dptr(out), _dptr(lse), _dptr(visited),
                                              _dptr(ws), ws_bytes, _stream(stream))
+
+    def prefill_append(self, layer, seq_ids, q_start, q_len, q, k_new, v_new, scale, out, lse, visited, ws,
+                       ws_bytes, stream=None) -> int:
+        s, qs, ql = _i32(seq_ids), _i32(q_start), _i32(q_len)
+        return lib().segkv_prefill_append(self.h, layer, len(s), _p(s), _p(qs), _p(ql), _dptr(q), _dptr(k_new),
+                                          _dptr(v_new), float(scale), _dptr(out), _dptr(lse), _dptr(visited),
+                                          _dptr(ws), ws_bytes, _stream(stream))
 
     def decode(self, layer, seq_ids, q_pos, q, scale, num_splits, out, lse, visited, ws, ws_bytes,
                stream=None) -> int:
@@ -298,6 +306,18 @@ class SegKV:
         lse = lse if lse is not None else t.empty((T, self.hq), dtype=t.float32, device=self.device)
         _check(self.handle.prefill_2src(layer, seq_ids, q_start, q_len, q, k_chunk, v_chunk, scale, out, lse,
                                         visited, self.ws, self.ws_bytes), "segkv_prefill_attn_2src", self.handle.h)
+        return out, lse
+
+    def prefill_append(self, layer: int, seq_ids, q_start, q_len, q, k_new, v_new, *, out=None, lse=None,
+                       visited=None, scale: float = 0.0):
+        """segkv_prefill_append: appends k_new / v_new [sum(q_len), Hkv, D] at q_start and attends
+        the range's queries, in one kernel (the kernel stores each page it loads)."""
+        t = self.torch
+        T = int(np.sum(q_len))
+        out = out if out is not None else t.empty((T, self.hq, self.d), dtype=t.bfloat16, device=self.device)
+        lse = lse if lse is not None else t.empty((T, self.hq), dtype=t.float32, device=self.device)
+        _check(self.handle.prefill_append(layer, seq_ids, q_start, q_len, q, k_new, v_new, scale, out, lse, visited,
+                                          self.ws, self.ws_bytes), "segkv_prefill_append", self.handle.h)
         return out, lse
 
     def decode(self, layer: int, seq_ids, q_pos, q, *, out=None, lse=None, visited=None, scale: float = 0.0,

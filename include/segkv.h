@@ -164,6 +164,28 @@ int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, 
                        uint64_t *visited, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Fused append + prefill: the result of segkv_append (start_pos = q_start_pos, num_new =
+ * q_len, K/V = k_new / v_new) followed by segkv_prefill_attn over the appended range, in one
+ * kernel.  The keys of the range come from k_new / v_new as in segkv_prefill_attn_2src; once a
+ * page of them has landed in shared memory, the work item whose query range holds the page's
+ * first position also writes it to its pool page (a TMA store from shared memory) and records
+ * it in the page table, so the append costs no kernel of its own (per-head storage grown as
+ * it is attended: zhichai.net news item "What Happened", item 3).  Page tables, the cursor,
+ * lengths, out, lse and visited equal those of the two calls; rows of a sequence's last page
+ * past its last token hold finite values (the next packed sequence's rows, or zeros) where
+ * segkv_append writes zeros -- no attention ever reads them unmasked.  Requires
+ * q_start_pos[b] == segkv_seq_len(h, layer, seq_ids[b]), a multiple of the page size, and
+ * (local heads) that the ring still holds every key the range's queries need after the
+ * append (the condition of segkv_prefill_attn).  While a page is shared after a fork the call
+ * runs as segkv_append then segkv_prefill_attn.
+ * Errors: INVALID_ARG, RING_TOO_SMALL, OUT_OF_PAGES (nothing changed), WORKSPACE, CUDA.
+ */
+int segkv_prefill_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                         const int32_t *q_len, const void *q, const void *k_new, const void *v_new,
+                         float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/*
  * Two-source prefill: the same attention as segkv_prefill_attn for a chunk that is NOT yet
  * appended.  The keys of each sequence's query range come from k_chunk / v_chunk (DEVICE
  * bf16 [sum(q_len), Hkv, D], packed like q); only the context before the range is read from

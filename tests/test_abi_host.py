@@ -178,3 +178,16 @@ def test_two_source_prefill_validation_happens_before_any_enqueue():
     assert h.prefill_2src(0, [0], [0], [10], FAKE, FAKE + 4, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
     # past max_seq_len
     assert h.prefill_2src(0, [0], [0], [4097], FAKE, FAKE, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+
+
+def test_fused_prefill_append_validation_happens_before_any_enqueue():
+    h = handle()
+    big = 1 << 20
+    # not at the sequence's end, not page-aligned, missing or misaligned K/V, past max_seq_len
+    assert h.prefill_append(0, [0], [64], [10], FAKE, FAKE, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.prefill_append(0, [0], [0], [10], FAKE, 0, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.prefill_append(0, [0], [0], [10], FAKE, FAKE, FAKE + 4, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    assert h.prefill_append(0, [0], [0], [4097], FAKE, FAKE, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 1
+    # the default ring (13 pages of 64) cannot hold a 1000-token chunk's windows after it
+    assert h.prefill_append(0, [0], [0], [1000], FAKE, FAKE, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 4
+    assert h.seq_len(0, 0) == 0 and h.pages_used == 0

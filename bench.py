@@ -301,7 +301,7 @@ def main():
     # (segkv_prefill_append: the prefill kernel also stores the K/V pages it loads) is timed
     # afterwards for comparison.
     def fused():
-        kv.prefill_append(0, [0], [0], [L], q_d, k_d, v_d, out=out, lse=lse, visited=visited)
+        kv.prefill_append(0, [0], [0], [L], q_d, k_d, v_d, out=out, lse=lse)
 
     def step():
         kv.handle.reset(stream)

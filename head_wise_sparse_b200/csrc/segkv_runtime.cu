@@ -13,7 +13,6 @@
 #include <cstring>
 #include <new>
 #include <string>
-#include <unordered_map>
 #include <utility>
 #include <vector>
 
@@ -81,6 +80,7 @@ struct segkv {
   // the host plan every allocation, including the copies on write after a fork.
   std::vector<int32_t> slot_k;  // [layers * max_seqs * hkv * max_lp]
   std::vector<int32_t> ref;     // [num_pages]
+  std::vector<int32_t> ref_scratch;  // [num_pages]: a call's pending reference-count changes, 0 between calls
   long long n_shared = 0;       // entries with ref >= 2: while 0, no append copies a page
   int ring = 0, max_lp = 0, G = 0;
   long long pages_used = 0;
@@ -478,6 +478,7 @@ int segkv_create(const segkv_config *c, segkv_t **out) {
   h->len.assign((size_t)c->num_layers * c->max_seqs, 0);
   h->slot_k.assign((size_t)c->num_layers * c->max_seqs * c->num_kv_heads * h->max_lp, -1);
   h->ref.assign((size_t)c->num_pages, 0);
+  h->ref_scratch.assign((size_t)c->num_pages, 0);
   h->cfg.head_class = nullptr;
   *out = h;
   return SEGKV_OK;
@@ -605,11 +606,14 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
   // changes to the mirror, applied once the call is accepted; refcounts seen through them, so
   // a page one sequence of the call copies is no longer shared for a later one
   std::vector<std::pair<size_t, int32_t>> slot_set;
-  std::unordered_map<int32_t, int32_t> ref_delta;
-  auto ref_of = [&](int32_t k) {
-    const auto it = ref_delta.find(k);
-    return h->ref[k] + (it == ref_delta.end() ? 0 : it->second);
-  };
+  std::vector<int32_t> ref_keys;  // entries whose count the call changes (pending in ref_scratch)
+  struct ScratchClear {           // every exit leaves ref_scratch all zero again
+    std::vector<int32_t> &scratch, &keys;
+    ~ScratchClear() {
+      for (const int32_t k : keys) scratch[k] = 0;
+    }
+  } scratch_clear{h->ref_scratch, ref_keys};
+  auto ref_of = [&](int32_t k) { return h->ref[k] + h->ref_scratch[k]; };
   long long new_pages = 0;
   for (int b = 0; b < nseq; ++b)
     for (int k = 0; k < H; ++k) {
@@ -637,7 +641,10 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
         plan.push_back(k_new);
         if (copy_rows > 0) jobs.push_back(make_int4(k_new, k_old, copy_rows, 0));
         slot_set.push_back({idx, k_new});
-        if (k_old >= 0) ref_delta[k_old] -= 1;
+        if (k_old >= 0) {
+          if (h->ref_scratch[k_old] == 0) ref_keys.push_back(k_old);
+          h->ref_scratch[k_old] -= 1;
+        }
       }
     }
   pair_page[(size_t)nseq * H] = (int32_t)plan.size();
@@ -678,10 +685,10 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
       h->slot_k[e.first] = e.second;
       h->ref[e.second] = 1;
     }
-    for (const auto &e : ref_delta) {
-      const int32_t before = h->ref[e.first];
-      h->ref[e.first] += e.second;
-      if (before >= 2 && h->ref[e.first] < 2) h->n_shared--;
+    for (const int32_t k : ref_keys) {
+      const int32_t before = h->ref[k];
+      h->ref[k] += h->ref_scratch[k];
+      if (before >= 2 && h->ref[k] < 2) h->n_shared--;
     }
   } else {  // the kernel's closed form: new pages in the allocation order
     int32_t k_new = (int32_t)h->pages_used;

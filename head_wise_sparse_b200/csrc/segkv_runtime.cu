@@ -1061,14 +1061,14 @@ int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
   int chunks = 1;
   for (const int4 &it : items) chunks = std::max(chunks, ((int)((uint32_t)it.w >> 20)) + 1);
   const int slots = kRouterColGroups * chunks;
-  {
-    std::vector<size_t> order(items.size());
-    for (size_t i = 0; i < order.size(); ++i) order[i] = i;
-    std::stable_sort(order.begin(), order.end(), [&](size_t x, size_t y) {
-      return (items[x].w & 0xFFFFF) > (items[y].w & 0xFFFFF);
-    });
+  {  // longest first, equal lengths in creation order: a counting sort on the tile count
+    int max_nt = 0;
+    for (const int4 &it : items) max_nt = std::max(max_nt, it.w & 0xFFFFF);
+    std::vector<int32_t> start((size_t)max_nt + 2, 0);
+    for (const int4 &it : items) ++start[(size_t)(max_nt - (it.w & 0xFFFFF)) + 1];
+    for (size_t v = 1; v < start.size(); ++v) start[v] += start[v - 1];
     std::vector<int4> sorted(items.size());
-    for (size_t i = 0; i < order.size(); ++i) sorted[i] = items[order[i]];
+    for (const int4 &it : items) sorted[(size_t)start[(size_t)(max_nt - (it.w & 0xFFFFF))]++] = it;
     items.swap(sorted);
   }
   const size_t items_off = align_up(kHeaderBytes + sizeof(RouterSeq) * nseq, 16);

@@ -101,8 +101,10 @@ def _i32(x) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
 
 
-def _p(a: np.ndarray):
-    return a.ctypes.data_as(ctypes.c_void_p)
+def _p(a: np.ndarray) -> int:
+    # the address as a plain int (data_as builds a ctypes object per call, several times
+    # slower); the caller keeps `a` alive for the duration of the call
+    return a.ctypes.data
 
 
 def _dptr(t) -> Optional[int]:
@@ -132,7 +134,7 @@ class Handle:
                  state):
         self._cls = np.ascontiguousarray(np.asarray(head_class, dtype=np.uint8).reshape(-1))
         self.cfg = Config(num_layers, num_q_heads, num_kv_heads, head_dim, page_size, window, ring_pages, max_seqs,
-                          max_seq_len, max_chunk, _p(self._cls).value, num_pages, _dptr(k_pool), _dptr(v_pool),
+                          max_seq_len, max_chunk, _p(self._cls), num_pages, _dptr(k_pool), _dptr(v_pool),
                           _dptr(page_table), _dptr(free_list), _dptr(state))
         self.h = ctypes.c_void_p()
         _check(lib().segkv_create(ctypes.byref(self.cfg), ctypes.byref(self.h)), "segkv_create")

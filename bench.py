@@ -61,6 +61,29 @@ def visible_pairs(w: wl.Workload, layer: int = 0) -> int:
     return n
 
 
+def rank_tools(torch, dist, device):
+    """(barrier, max_over_ranks) for one process per GPU: a no-op and the identity on one
+    rank; else a process-group barrier and an all-reduce MAX of a float64 on `device` (the
+    GPU under NCCL, the CPU under gloo).  Every multi-GPU time is the slowest rank's."""
+    if dist is None:
+        return (lambda: None), (lambda x: x)
+
+    def barrier():
+        dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
+def whole_job(units_per_rank: float, world: int, t_max_ms: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (t_max_ms * 1e-3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -263,16 +286,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = rank_tools(torch, dist if world > 1 else None, dev)
 
     pk, pk_src = peaks()
     stream = torch.cuda.current_stream()

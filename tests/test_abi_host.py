@@ -191,3 +191,15 @@ def test_fused_prefill_append_validation_happens_before_any_enqueue():
     # the default ring (13 pages of 64) cannot hold a 1000-token chunk's windows after it
     assert h.prefill_append(0, [0], [0], [1000], FAKE, FAKE, FAKE, 0.0, FAKE, FAKE, 0, FAKE, big, stream=0) == 4
     assert h.seq_len(0, 0) == 0 and h.pages_used == 0
+
+
+def test_binding_argument_counts_match_the_header():
+    # every declaration's parameter count equals the binding's ctypes signature, so a change
+    # to include/segkv.h that the binding missed fails here rather than on a GPU
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    lib = segkv.lib()
+    for name, params in re.findall(r"\b(segkv_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text):
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        argtypes = getattr(lib, name).argtypes
+        if argtypes is not None:
+            assert len(argtypes) == n, (name, len(argtypes), n)

@@ -15,7 +15,7 @@
  *   - attention for every head runs over that head's own pages; the result equals plain
  *     masked softmax attention with an explicit per-head visibility row.
  *
- * Readings taken where the pages are silent (each listed in the design doc):
+ * Readings taken where the pages are silent:
  *   visibility of a query at position p:  global  k <= p;   local  p - W < k <= p;
  *   query head h reads KV head h / G (G = Hq / Hkv, contiguous groups);
  *   lse = natural log of the sum of exp(scale * q.k) over visible keys;

@@ -1,15 +1,17 @@
 #!/usr/bin/env python
 """Benchmark of the segmented paged attention hot path on B200.
 
-One step = one prefill of the Mistral-7B-shaped single-layer workload (L = 8192, Hq 32,
-Hkv 8, D 128, one global KV head, seven local heads with W = 1024, 64-token pages,
-shuffled physical pages): empty the cache, append the 8192 tokens' K/V into every head's
-own pages (page-table build + scatter), and run the causal varlen prefill over those pages.
-Metric: TFLOP/s over visible (q, k) pairs, FLOPs = 4 * D * sum of visible pairs.
+One step = the Llama-3.3-70B-shaped varlen prefill over 4 layers (4 sequences of seeded
+lengths in [8192, 32768], Hq 64, Hkv 8, D 128, per layer one global KV head and seven local
+heads with W = 2048, 64-token pages, shuffled physical pages): empty the cache, append every
+layer's K/V into each head's own pages (page-table build + scatter), and run the causal
+varlen prefill of every layer over those pages.  Metric: TFLOP/s over visible (q, k) pairs,
+FLOPs = 4 * D * sum of visible pairs over the 4 layers.
 
-The same JSON line carries a ``decode`` object: the batched-decode workload (64 sequences
-at 32K context, Hq 64, Hkv 8, one global head, W = 4096 rings of 65 pages): per step, the
-append of one new token per sequence plus split-K decode and the LSE combine, in KV GB/s.
+The same JSON line carries the other workloads as sub-objects, each with its own roofline:
+the Mistral-7B-shaped single-layer prefill, the 128K-context chunked prefill (one-source and
+two-source), the tiny prefill, the KV append on three shapes, the batched decode step (64
+sequences at 32K, KV GB/s), attention as a router, query relocation and copy on write.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl segkv|reference]
 
@@ -39,13 +41,16 @@ sys.path.insert(0, ROOT)
 from head_wise_sparse_b200 import workloads as wl  # noqa: E402
 
 METRIC = "prefill TFLOP/s over visible (q,k) pairs (% BF16 peak); decode KV GB/s (% HBM)"
+HEADLINE = "llama70b_varlen_prefill_4x4layers"
 PREFILL = "mistral7b_prefill_L8192"
+TINY = "tiny_prefill_L1024_D64"
 DECODE = "decode_64x32k"
 CHUNKED = "mha_chunked_prefill_128k"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_SOURCES = ["head_wise_sparse_b200/csrc/prefill_sm100.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 DECODE_SOURCES = ["head_wise_sparse_b200/csrc/decode.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 ROUTER_SOURCES = ["head_wise_sparse_b200/csrc/router_sm100.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
+APPEND_SOURCES = ["head_wise_sparse_b200/csrc/storage.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -224,7 +229,7 @@ def run_reference(args):
     import oracle as orc
     from tests.harness import oracle_replay, q_for_call, step_queries
 
-    w = wl.CONFIGS[PREFILL]
+    w = wl.CONFIGS[HEADLINE]
     o = orc.Oracle.for_workload(w)
     oracle_replay(w, 0, o)
     ids, qs, ql = step_queries(w)
@@ -249,7 +254,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / max(args.steps, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": PREFILL, "sample": "rows"},
+        "config": {"workload": HEADLINE, "sample": "rows"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": orc.host_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -259,63 +264,171 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------- GPU arm
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--impl", default="segkv", choices=["segkv", "reference"])
-    ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-    if args.impl == "reference":
-        return run_reference(args)
-
-    import torch
-    import torch.distributed as dist
-
+def new_handle(w: wl.Workload, dev, *, ring=None, max_chunk=None, ws_batch=None, ws_tokens=None, max_seqs=None,
+               free_list=None, num_pages=None, max_seq_len=None):
     from head_wise_sparse_b200.segkv import SegKV
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    return SegKV(num_layers=w.layers, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=w.page,
+                 window=w.window, head_class=w.class_array(), num_pages=num_pages or w.num_pages,
+                 free_list=w.free_list() if free_list is None else free_list, max_seqs=max_seqs or len(w.seqs),
+                 max_seq_len=max_seq_len or w.max_seq_len, ring_pages=ring or w.ring_pages,
+                 max_chunk=max_chunk or w.max_chunk, ws_batch=ws_batch or len(w.seqs),
+                 ws_tokens=ws_tokens or max(sum(s.q_hi - s.q_lo for s in w.seqs), 1), device=dev)
 
-    barrier, max_over_ranks = rank_tools(torch, dist if world > 1 else None, dev)
 
-    pk, pk_src = peaks()
-    stream = torch.cuda.current_stream()
+def events(torch, n, k):
+    return [[torch.cuda.Event(enable_timing=True) for _ in range(k)] for _ in range(n)]
 
-    # ------------------------------------------------------------------ prefill workload
+
+def mean_ms(evs, a, b):
+    return sum(e[a].elapsed_time(e[b]) for e in evs) / len(evs)
+
+
+def roofline(achieved, peak, unit, bound, kernel, traffic=None, **extra):
+    r = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+         "traffic": traffic, "kernel": kernel}
+    r.update(extra)
+    return r
+
+
+def append_bytes(w: wl.Workload, tokens: int) -> int:
+    """Algorithmic bytes of appending `tokens` tokens: K and V rows read and written once."""
+    return 2 * 2 * tokens * w.hkv * w.d * 2
+
+
+def bench_headline(args, torch, dev, stream, barrier, max_over_ranks, world, pk, sampler):
+    """The Llama-3.3-70B-shaped varlen prefill over 4 layers: reset + 4 appends + 4 prefills."""
+    w = wl.CONFIGS[HEADLINE]
+    lens = [s.length for s in w.seqs]
+    ids, starts, T = list(range(len(lens))), [0] * len(lens), int(sum(lens))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3)
+    # seeded N(0, 1) inputs drawn on the device (the workload's distribution; the parity tests
+    # use the workload's own bit patterns)
+    q = [torch.randn((T, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16) for _ in range(w.layers)]
+    k = [torch.randn((T, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16) for _ in range(w.layers)]
+    v = [torch.randn((T, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16) for _ in range(w.layers)]
+    out = [torch.empty((T, w.hq, w.d), dtype=torch.bfloat16, device=dev) for _ in range(w.layers)]
+    lse = [torch.empty((T, w.hq), dtype=torch.float32, device=dev) for _ in range(w.layers)]
+    vis = torch.zeros((w.layers, len(ids), w.hq), dtype=torch.int64, device=dev)
+    kv = new_handle(w, dev, ws_tokens=T, max_chunk=max(lens))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    pairs = [visible_pairs(w, l) for l in range(w.layers)]
+    flops = 4.0 * w.d * sum(pairs)
+    L = w.layers
+
+    def step(ev=None, with_vis=False):
+        if ev:
+            ev[0].record(stream)
+        kv.handle.reset(stream)
+        for l in range(L):
+            kv.append(l, ids, starts, lens, k[l], v[l])
+        if ev:
+            ev[1].record(stream)
+        for l in range(L):
+            kv.prefill(l, ids, starts, lens, q[l], out=out[l], lse=lse[l], visited=vis[l] if with_vis else None)
+            if ev:
+                ev[2 + l].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    ev = events(torch, args.steps, 2 + L)
+    vis.zero_()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = sampler.mark()
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)  # evict L2 between timed steps (not timed)
+        step(ev[s], with_vis=True)
+    torch.cuda.synchronize()
+    barrier()
+    t1 = sampler.mark()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    # the kernel's own count of visited pairs (columns its masks kept) must equal the closed form
+    got = vis.sum(dim=(1, 2)).cpu().numpy()
+    for l in range(L):
+        if int(got[l]) != args.steps * pairs[l]:
+            raise RuntimeError(f"layer {l}: visited pairs {int(got[l])} != {args.steps} x {pairs[l]}")
+    t_step = max_over_ranks(mean_ms(ev, 0, 2 + L - 1))
+    t_app = max_over_ranks(mean_ms(ev, 0, 1))
+    t_pre = max_over_ranks(sum(mean_ms(ev, 1 + l, 2 + l) for l in range(L)))
+    achieved = flops / (t_pre * 1e-3) / 1e12
+    app_b = L * append_bytes(w, T)
+
+    # ------------------------------------------------------------------ end to end, host buffers
+    # every step copies all 4 layers' Q, K and V in from pinned host memory and every layer's
+    # output and lse back out
+    q_h = [t.to("cpu").pin_memory() for t in q]
+    k_h = [t.to("cpu").pin_memory() for t in k]
+    v_h = [t.to("cpu").pin_memory() for t in v]
+    out_h = [torch.empty((T, w.hq, w.d), dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+    lse_h = [torch.empty((T, w.hq), dtype=torch.float32).pin_memory() for _ in range(L)]
+    e2e_steps = max(3, min(args.steps, 8))
+    ev2 = events(torch, e2e_steps, 2)
+    barrier()
+    torch.cuda.synchronize()
+    for s in range(e2e_steps):
+        flush.fill_(s & 0xFF)
+        ev2[s][0].record(stream)
+        for l in range(L):
+            q[l].copy_(q_h[l], non_blocking=True)
+            k[l].copy_(k_h[l], non_blocking=True)
+            v[l].copy_(v_h[l], non_blocking=True)
+        step()
+        for l in range(L):
+            out_h[l].copy_(out[l], non_blocking=True)
+            lse_h[l].copy_(lse[l], non_blocking=True)
+        ev2[s][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_e2e = max_over_ranks(mean_ms(ev2, 0, 1))
+    h2d = sum(t.numel() * t.element_size() for t in q_h + k_h + v_h)
+    d2h = sum(t.numel() * t.element_size() for t in out_h + lse_h)
+    e2e = {"value": world * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e, "steps": e2e_steps}
+    res = {
+        "value": world * flops / (t_step * 1e-3) / 1e12, "ms_per_step": t_step, "prefill_kernel_ms": t_pre,
+        "append_ms": t_app, "flops_per_step": flops, "visible_pairs_per_layer": pairs, "e2e": e2e,
+        "roofline": roofline(achieved, pk["bf16_tflops"], "TFLOP/s", "tensor",
+                             "prefill_kernel<128> (events around the 4 segkv_prefill_attn calls of a step)",
+                             profiled_traffic("prefill_llama70b_varlen.md", PREFILL_SOURCES),
+                             peak_source="measured bf16 burst (cuBLAS)",
+                             frac_of_sustained=achieved / pk["bf16_tflops_sustained"]),
+        "append": {"bytes": app_b, "ms": t_app, "GB/s": app_b / (t_app * 1e-3) / 1e9,
+                   "roofline": roofline(app_b / (t_app * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
+                                        "reset_kernel + append_kernel x 4 (events around reset + the 4 segkv_append calls)")},
+        "config": {"workload": HEADLINE, "layers": L, "seq_lens": lens, "q_heads": w.hq, "kv_heads": w.hkv,
+                   "head_dim": w.d, "page_size": w.page, "window": w.window,
+                   "global_kv_heads_per_layer": [int(sum(c)) for c in w.classes],
+                   "step": "reset + append of 4 layers (page ids + scatter) + prefill of 4 layers",
+                   "l2": "inputs larger than L2 (1.4 GB of Q a layer); L2 also flushed between timed steps "
+                         "(256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world}", "global_batch": len(lens), "seq_len": max(lens)},
+        "gpu_launches": (1 + 2 * L) * args.steps,
+        "clock_window": (t0, t1),
+    }
+    del kv, q, k, v, out, lse, q_h, k_h, v_h, out_h, lse_h, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_mistral(args, torch, dev, stream, max_over_ranks, world, pk):
+    """The Mistral-7B-shaped single-layer step (reset + append + prefill), the same work as one
+    fused call, and the router and query relocation on the same queries."""
     w = wl.CONFIGS[PREFILL]
     L = w.seqs[0].length
-    q_bits = w.q(0, 0, 0, L)
-    k_bits = w.k(0, 0, 0, L)
-    v_bits = w.v(0, 0, 0, L)
-
-    def dev_bf16(bits):
-        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
-
-    q_d, k_d, v_d = dev_bf16(q_bits), dev_bf16(k_bits), dev_bf16(v_bits)
-    kv = SegKV(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=w.page, window=w.window,
-               head_class=w.class_array(), num_pages=w.num_pages, free_list=w.free_list(), max_seqs=1,
-               max_seq_len=L, ring_pages=w.ring_pages, max_chunk=L, ws_batch=1, ws_tokens=L, device=dev)
+    dev_bf16 = lambda bits: torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+    q_d, k_d, v_d = dev_bf16(w.q(0, 0, 0, L)), dev_bf16(w.k(0, 0, 0, L)), dev_bf16(w.v(0, 0, 0, L))
+    kv = new_handle(w, dev, ws_tokens=L, max_chunk=L)
     out = torch.empty((L, w.hq, w.d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((L, w.hq), dtype=torch.float32, device=dev)
     visited = torch.zeros((1, w.hq), dtype=torch.int64, device=dev)
     flops = 4.0 * w.d * visible_pairs(w)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
-
-    # The step: reset, segkv_append, segkv_prefill_attn.  The same work as one fused call
-    # (segkv_prefill_append: the prefill kernel also stores the K/V pages it loads) is timed
-    # afterwards for comparison.
-    def fused():
-        kv.prefill_append(0, [0], [0], [L], q_d, k_d, v_d, out=out, lse=lse)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def step():
         kv.handle.reset(stream)
@@ -325,122 +438,83 @@ def main():
         step()
         kv.prefill(0, [0], [0], [L], q_d, out=out, lse=lse, visited=visited)
     torch.cuda.synchronize()
-    if kv.device_status() != 0:
-        raise RuntimeError("device error word set during warm-up")
-    props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler(str(getattr(props, "uuid", "")))
-    time.sleep(0.3)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev = events(torch, args.steps, 4)
     visited.zero_()
-    barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
     for s in range(args.steps):
-        flush.fill_(s & 0xFF)  # evict L2 between timed steps (not timed)
+        flush.fill_(s & 0xFF)
         ev[s][0].record(stream)
-        step()
+        kv.handle.reset(stream)
         ev[s][1].record(stream)
-        kv.prefill(0, [0], [0], [L], q_d, out=out, lse=lse, visited=visited)
+        kv.append(0, [0], [0], [L], k_d, v_d)
         ev[s][2].record(stream)
+        kv.prefill(0, [0], [0], [L], q_d, out=out, lse=lse, visited=visited)
+        ev[s][3].record(stream)
     torch.cuda.synchronize()
-    barrier()
-    t_wall1 = time.time()
-    clocks = sampler.summary(t_wall0, t_wall1)
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the Mistral-shaped steps")
+    if int(visited.sum().item()) != args.steps * visible_pairs(w):
+        raise RuntimeError("Mistral-shaped visited pairs differ from the closed form")
+    t_step = max_over_ranks(mean_ms(ev, 0, 3))
+    t_app = max_over_ranks(mean_ms(ev, 1, 2))
+    t_pre = max_over_ranks(mean_ms(ev, 2, 3))
+    app_b = append_bytes(w, L)
     # the same work as one fused call: reset, then segkv_prefill_append
     for _ in range(args.warmup):
         kv.handle.reset(stream)
-        fused()
-    evf = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
+        kv.prefill_append(0, [0], [0], [L], q_d, k_d, v_d, out=out, lse=lse)
+    evf = events(torch, args.steps, 2)
     for s in range(args.steps):
         flush.fill_(s & 0xFF)
-        evf[s][0].record(stream)
         kv.handle.reset(stream)
+        evf[s][0].record(stream)
+        kv.prefill_append(0, [0], [0], [L], q_d, k_d, v_d, out=out, lse=lse)
         evf[s][1].record(stream)
-        fused()
-        evf[s][2].record(stream)
     torch.cuda.synchronize()
-    barrier()
-    tf_step = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in evf) / args.steps)
-    fused_call = {"value": world * flops / (tf_step * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": tf_step,
-                  "prefill_append_ms": max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in evf) / args.steps),
-                  "step": "reset + segkv_prefill_append (the prefill kernel stores the K/V pages it loads)",
-                  "gpu_launches": 2 * args.steps}
     if kv.device_status() != 0:
-        raise RuntimeError("device error word set during the timed steps")
-    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    pre_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    app_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    # the kernel's own count of visited pairs must equal the closed form
-    vis_total = int(visited.sum().item())
-    if vis_total != args.steps * visible_pairs(w):
-        raise RuntimeError(f"visited pairs {vis_total} != {args.steps} x {visible_pairs(w)}")
-    t_step = max_over_ranks(sum(step_ms) / args.steps)
-    t_pre = max_over_ranks(sum(pre_ms) / args.steps)
-    value = world * flops / (t_step * 1e-3) / 1e12
-    achieved = flops / (t_pre * 1e-3) / 1e12
-    traffic = profiled_traffic("prefill_mistral7b_L8192.md", PREFILL_SOURCES)
-
-    # ------------------------------------------------------------------ e2e through host buffers
-    q_h = torch.from_numpy(q_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    k_h = torch.from_numpy(k_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    v_h = torch.from_numpy(v_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    out_h = torch.empty_like(out, device="cpu").pin_memory()
-    lse_h = torch.empty_like(lse, device="cpu").pin_memory()
-    e2e_steps = min(args.steps, 30)
-    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
-    barrier()
-    torch.cuda.synchronize()
-    for s in range(e2e_steps):
-        flush.fill_(s & 0xFF)
-        ev2[s][0].record(stream)
-        q_d.copy_(q_h, non_blocking=True)
-        k_d.copy_(k_h, non_blocking=True)
-        v_d.copy_(v_h, non_blocking=True)
-        step()
-        kv.prefill(0, [0], [0], [L], q_d, out=out, lse=lse, visited=visited)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
-        ev2[s][1].record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    t_e2e = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2) / e2e_steps)
-    h2d = q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2
-    d2h = out_h.numel() * 2 + lse_h.numel() * 4
-    e2e = {"value": world * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e}
-    # ------------------------------------------------------------------ query relocation
-    # segkv_relocate_q on the same workload's queries (local heads turned by -delta, the
-    # global head copied): HBM-bound, one read and one write of every query element.
+        raise RuntimeError("device error word set during the fused calls")
+    t_fused = max_over_ranks(mean_ms(evf, 0, 1))
+    res = {
+        "workload": PREFILL, "value": world * flops / (t_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "ms_per_step": t_step, "prefill_kernel_ms": t_pre, "append_ms": t_app,
+        "step": "reset + append (page ids + scatter) + prefill",
+        "roofline": roofline(flops / (t_pre * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s", "tensor",
+                             "prefill_kernel<128> (events around segkv_prefill_attn: metadata upload + kernel)",
+                             profiled_traffic("prefill_mistral7b_L8192.md", PREFILL_SOURCES)),
+        "append": {"bytes": app_b, "ms": t_app,
+                   "roofline": roofline(app_b / (t_app * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
+                                        "append_kernel (events around segkv_append)",
+                                        profiled_traffic("append_mistral7b_L8192.md", APPEND_SOURCES))},
+        "fused_append_prefill": {"ms_per_call": t_fused, "value": world * flops / (t_fused * 1e-3) / 1e12,
+                                 "unit": "TFLOP/s", "two_call_ms": t_app + t_pre,
+                                 "step": "segkv_prefill_append (the prefill kernel stores the K/V pages it loads)"},
+        "gpu_launches": 3 * args.steps,
+    }
+    # query relocation: local heads turned by -delta, the global head copied (one read + one
+    # write of every query element)
     q_rel = torch.empty_like(q_d)
     shift = torch.full((L,), 100000, dtype=torch.int32, device=dev)
     for _ in range(args.warmup):
         kv.relocate_q(0, q_d, shift, out=q_rel)
-    evr = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(args.steps, 50))]
+    evr = events(torch, min(args.steps, 50), 2)
     for e in evr:
         flush.fill_(1)
         e[0].record(stream)
         kv.relocate_q(0, q_d, shift, out=q_rel)
         e[1].record(stream)
     torch.cuda.synchronize()
-    t_rel = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evr) / len(evr))
-    rel_bytes = 2 * q_d.numel() * 2
-    relocate = {"metric": "query relocation GB/s", "value": world * rel_bytes / (t_rel * 1e-3) / 1e9, "unit": "GB/s",
-                "ms_per_call": t_rel, "bytes_per_call": rel_bytes,
-                "roofline": {"bound": "hbm", "achieved": rel_bytes / (t_rel * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
-                             "unit": "GB/s", "frac": rel_bytes / (t_rel * 1e-3) / 1e9 / pk["hbm_gbs"], "traffic": None,
-                             "kernel": "relocate_q_kernel (events around segkv_relocate_q)"}}
-    # ------------------------------------------------------------------ attention as a router
-    # segkv_router_topk on the same queries and the last prefill's lse: every token's received
-    # attention mass and the top quarter of the tokens.  One exponential per visible pair on
-    # the MUFU bounds it (16 per clock per SM).
+    t_rel = max_over_ranks(mean_ms(evr, 0, 1))
+    rel_b = 2 * q_d.numel() * 2
+    res["relocate"] = {"metric": "query relocation GB/s", "value": world * rel_b / (t_rel * 1e-3) / 1e9,
+                       "unit": "GB/s", "ms_per_call": t_rel, "bytes_per_call": rel_b,
+                       "roofline": roofline(rel_b / (t_rel * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
+                                            "relocate_q_kernel (events around segkv_relocate_q)")}
+    # attention as a router: every token's received attention mass and the top quarter
     k_top = [L // 4]
     rt_scores = torch.empty((L,), dtype=torch.float32, device=dev)
     rt_rows = torch.empty((L // 4,), dtype=torch.int32, device=dev)
     for _ in range(args.warmup):
         kv.router_topk(0, [0], [0], [L], q_d, lse, k_top, scores=rt_scores, rows=rt_rows)
-    evt = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(args.steps, 50))]
+    evt = events(torch, min(args.steps, 50), 2)
     for e in evt:
         flush.fill_(2)
         e[0].record(stream)
@@ -449,55 +523,118 @@ def main():
     torch.cuda.synchronize()
     if kv.device_status() != 0:
         raise RuntimeError("device error word set during the router benchmark")
-    t_rt = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evt) / len(evt))
+    t_rt = max_over_ranks(mean_ms(evt, 0, 1))
     pairs = visible_pairs(w)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    max_mhz = float((clocks or {}).get("sm_max_mhz") or 1965.0)  # the GPU's maximum SM clock (nvidia-smi)
-    mufu_peak = 16 * sms * max_mhz * 1e6 / 1e9  # G exponentials per second at that clock
-    router = {"metric": "router visible pairs/s", "value": world * pairs / (t_rt * 1e-3) / 1e9, "unit": "Gpair/s",
-              "ms_per_call": t_rt, "pairs_per_call": pairs, "k": k_top[0],
-              "step": "segkv_router_topk: received attention mass of 8192 tokens (32 query heads) + top 2048",
-              "roofline": {"bound": "alu", "achieved": pairs / (t_rt * 1e-3) / 1e9, "peak": mufu_peak,
-                           "unit": "Gexp/s", "frac": pairs / (t_rt * 1e-3) / 1e9 / mufu_peak,
-                           "traffic": profiled_traffic("router_mistral7b_L8192.md", ROUTER_SOURCES),
-                           "peak_source": f"MUFU ex2: 16 per clock per SM x {sms} SMs x {max_mhz:.0f} MHz",
-                           "kernel": "router_kernel<128> + score_sum_kernel + topk_kernel (events around segkv_router_topk)"},
-              "gpu_launches": 3 * len(evt)}
+    mufu_peak = 16 * sms * 1965.0 * 1e6 / 1e9  # G exponentials per second at the maximum SM clock
+    res["router"] = {"metric": "router visible pairs/s", "value": world * pairs / (t_rt * 1e-3) / 1e9,
+                     "unit": "Gpair/s", "ms_per_call": t_rt, "pairs_per_call": pairs, "k": k_top[0],
+                     "step": "segkv_router_topk: received attention mass of 8192 tokens (32 query heads) + top 2048",
+                     "roofline": roofline(pairs / (t_rt * 1e-3) / 1e9, mufu_peak, "Gexp/s", "alu",
+                                          "router_kernel<128> + score_sum_kernel + topk_kernel (events around "
+                                          "segkv_router_topk)",
+                                          profiled_traffic("router_mistral7b_L8192.md", ROUTER_SOURCES),
+                                          peak_source=f"MUFU ex2: 16 per clock per SM x {sms} SMs x 1965 MHz "
+                                                      "(the maximum SM clock)"),
+                     "gpu_launches": 3 * len(evt)}
     del kv, flush, q_rel
     torch.cuda.empty_cache()
+    return res
 
-    # ------------------------------------------------------------------ decode workload
-    decode = None
-    if not args.no_decode:
-        decode = bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk)
 
+def bench_tiny(args, torch, dev, stream, max_over_ranks, world, pk):
+    """The tiny prefill (L 1024, Hq 8, Hkv 4, D 64, page 16): a correctness-sized workload whose
+    whole run is shorter than a kernel launch's fixed costs."""
+    w = wl.CONFIGS[TINY]
+    L = w.seqs[0].length
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1)
+    k = torch.randn((L, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn((L, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    kv = new_handle(w, dev, ws_tokens=L, max_chunk=L)
+    kv.append(0, [0], [0], [L], k, k)
+    out = torch.empty((L, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((L, w.hq), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        kv.prefill(0, [0], [0], [L], q, out=out, lse=lse)
+    ev = events(torch, args.steps, 2)
+    for e in ev:
+        e[0].record(stream)
+        kv.prefill(0, [0], [0], [L], q, out=out, lse=lse)
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the tiny prefill")
+    t = max_over_ranks(mean_ms(ev, 0, 1))
+    flops = 4.0 * w.d * visible_pairs(w)
+    del kv
+    return {"workload": TINY, "value": world * flops / (t * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_call": t,
+            "roofline": roofline(flops / (t * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s", "tensor",
+                                 "prefill_kernel<64> (events around segkv_prefill_attn); launch- and latency-bound"),
+            "gpu_launches": len(ev)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="segkv", choices=["segkv", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--headline-only", action="store_true", help="only the headline workload (for profiling)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    barrier, max_over_ranks = rank_tools(torch, dist if world > 1 else None, dev)
+    pk, pk_src = peaks()
+    stream = torch.cuda.current_stream()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(str(getattr(props, "uuid", "")))
+    time.sleep(0.3)
+
+    head = bench_headline(args, torch, dev, stream, barrier, max_over_ranks, world, pk, sampler)
+    t0, t1 = head.pop("clock_window")
+    clocks = sampler.summary(t0, t1)
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": PREFILL, "seq_len": L, "q_heads": w.hq, "kv_heads": w.hkv, "head_dim": w.d,
-                   "page_size": w.page, "window": w.window, "global_kv_heads": int(sum(w.classes[0])),
-                   "visible_pairs": visible_pairs(w), "step": "reset + append (page ids + scatter) + prefill",
-                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
-                   "parallelism": f"replicas x{world}"},
-        "prefill_kernel_ms": t_pre, "append_ms": max_over_ranks(sum(app_ms) / args.steps),
-        "fused_append_prefill": fused_call,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
-                     "peak_source": f"{pk_src} bf16 burst",
-                     "kernel": "prefill_kernel<128> (events around segkv_prefill_attn: metadata upload + kernel)"},
-        "e2e": e2e,
-        "gpu_launches": 3 * args.steps,
-        "clocks": clocks,
+        "metric": METRIC, "value": head["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) drawn on the device)",
+        "config": head["config"], "prefill_kernel_ms": head["prefill_kernel_ms"], "append_ms": head["append_ms"],
+        "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": clocks,
+        "peaks": {"source": pk_src, **pk},
     }
-    line["relocate"] = relocate
-    line["router"] = router
-    line["fork"] = bench_fork(args, torch, dev, stream, max_over_ranks, world, pk)
-    line["two_source"] = bench_two_source(args, torch, dev, stream, max_over_ranks, world, pk)
-    if decode is not None:
-        line["decode"] = decode
+    appends = {"llama70b_4_layers": head["append"]}
+    if not args.headline_only:
+        mis = bench_mistral(args, torch, dev, stream, max_over_ranks, world, pk)
+        appends["mistral7b"] = mis.pop("append")
+        line["relocate"] = mis.pop("relocate")
+        line["router"] = mis.pop("router")
+        line["fused_append_prefill"] = mis.pop("fused_append_prefill")
+        line["mistral7b"] = mis
+        chunk = bench_chunked(args, torch, dev, stream, max_over_ranks, world, pk)
+        appends["chunk_128k"] = chunk.pop("append")
+        line["chunked_128k"] = chunk
+        line["tiny"] = bench_tiny(args, torch, dev, stream, max_over_ranks, world, pk)
+        line["fork"] = bench_fork(args, torch, dev, stream, max_over_ranks, world, pk)
+        if not args.no_decode:
+            line["decode"] = bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk)
+    line["append"] = appends
     if rank == 0 and world == 1 and not args.no_cpu:
-        v_cpu, cores, desc = cpu_baseline(w, budget_s=3 * args.cpu_seconds, min_s=args.cpu_seconds)
+        v_cpu, cores, desc = cpu_baseline(wl.CONFIGS[HEADLINE], budget_s=3 * args.cpu_seconds, min_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
     if world > 1:
         dist.destroy_process_group()
@@ -506,33 +643,28 @@ def main():
     return 0
 
 
-def bench_two_source(args, torch, dev, stream, max_over_ranks, world, pk):
+def bench_chunked(args, torch, dev, stream, max_over_ranks, world, pk):
     """Chunked prefill of the 128K-context MHA workload (4096 queries at 126976, W 4096, P 64,
-    4 global + 28 local KV heads): segkv_prefill_attn_2src before the chunk is appended, with
-    local rings of ceil((W - 1) / P) + 1 = 65 pages, against segkv_prefill_attn after the
-    append, which needs 129.  Same keys, same FLOPs; the rings hold half the pages."""
-    from head_wise_sparse_b200.segkv import SegKV
-
+    4 global + 28 local KV heads): segkv_prefill_attn after the chunk is appended (local rings
+    of 129 pages), segkv_prefill_attn_2src before it is appended (rings of
+    ceil((W - 1) / P) + 1 = 65 pages: same keys, same FLOPs), and the append of the 4096-token
+    chunk itself (into an emptied handle, so every page is a new one)."""
     w = wl.CONFIGS[CHUNKED]
     s = w.seqs[0]
     ctx, C = s.context, s.new
     r_two = -(-(w.window - 1) // w.page) + 1
-    handles = {}
-    for name, ring in (("one", w.ring_pages), ("two", r_two)):
-        handles[name] = SegKV(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=w.page,
-                              window=w.window, head_class=w.class_array(), num_pages=w.num_pages,
-                              free_list=w.free_list(), max_seqs=1, max_seq_len=w.max_seq_len, ring_pages=ring,
-                              max_chunk=C, ws_batch=1, ws_tokens=C, device=dev)
+    handles = {name: new_handle(w, dev, ring=ring, max_chunk=C, ws_tokens=C)
+               for name, ring in (("one", w.ring_pages), ("two", r_two))}
     gen = torch.Generator(device=dev)
     gen.manual_seed(12)
     for lo in range(0, ctx, 4096):
         n = min(4096, ctx - lo)
-        k = (torch.randn((n, w.hkv, w.d), generator=gen, device=dev) / np.sqrt(w.d)).to(torch.bfloat16)
+        k = torch.randn((n, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
         v = torch.randn((n, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
         for kv in handles.values():
             kv.append(0, [0], [lo], [n], k, v)
         del k, v
-    kc = (torch.randn((C, w.hkv, w.d), generator=gen, device=dev) / np.sqrt(w.d)).to(torch.bfloat16)
+    kc = torch.randn((C, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
     vc = torch.randn((C, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
     q = torch.randn((C, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
     out = torch.empty((C, w.hq, w.d), dtype=torch.bfloat16, device=dev)
@@ -545,34 +677,60 @@ def bench_two_source(args, torch, dev, stream, max_over_ranks, world, pk):
     for name, call in calls.items():
         for _ in range(args.warmup):
             call()
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(args.steps, 20))]
+        ev = events(torch, min(args.steps, 20), 2)
         for e in ev:
             flush.fill_(3)
             e[0].record(stream)
             call()
             e[1].record(stream)
         torch.cuda.synchronize()
-        ms[name] = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev))
+        ms[name] = max_over_ranks(mean_ms(ev, 0, 1))
     handles["two"].append(0, [0], [ctx], [C], kc, vc)
     torch.cuda.synchronize()
     for kv in handles.values():
         if kv.device_status() != 0:
-            raise RuntimeError("device error word set during the two-source benchmark")
+            raise RuntimeError("device error word set during the chunked-prefill benchmark")
+    del handles
+    # the chunk's append: 4096 tokens x 32 heads into new pages of an emptied handle
+    kv = new_handle(w, dev, ring=w.ring_pages, max_chunk=C, ws_tokens=C)
+    app = []
+    for i in range(args.warmup + min(args.steps, 20)):
+        kv.handle.reset(stream)
+        flush.fill_(4)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kv.append(0, [0], [0], [C], kc, vc)
+        e1.record(stream)
+        if i >= args.warmup:
+            app.append((e0, e1))
+    torch.cuda.synchronize()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the chunk append")
+    t_app = max_over_ranks(sum(a.elapsed_time(b) for a, b in app) / len(app))
+    app_b = append_bytes(w, C)
+    del kv, flush
+    torch.cuda.empty_cache()
     flops = 4.0 * w.d * visible_pairs(w)
     n_local = int(w.hkv - sum(w.classes[0]))
     page_bytes = 2 * w.page * w.d * 2
-    res = {"workload": CHUNKED, "metric": "two-source chunked prefill TFLOP/s", "unit": "TFLOP/s",
-           "value": world * flops / (ms["two"] * 1e-3) / 1e12, "ms_per_call": ms["two"],
-           "one_source_ms_per_call": ms["one"], "ring_pages": {"two_source": r_two, "one_source": w.ring_pages},
-           "local_ring_bytes_saved_per_sequence": n_local * (w.ring_pages - r_two) * page_bytes,
-           "roofline": {"bound": "tensor", "achieved": flops / (ms["two"] * 1e-3) / 1e12, "peak": pk["bf16_tflops"],
-                        "unit": "TFLOP/s", "frac": flops / (ms["two"] * 1e-3) / 1e12 / pk["bf16_tflops"],
-                        "traffic": None, "kernel": "prefill_kernel<128>, chunk pages from the call's K/V "
-                                                   "(events around segkv_prefill_attn_2src)"},
-           "gpu_launches": 2 * len(ev)}
-    del handles, flush
-    torch.cuda.empty_cache()
-    return res
+    return {
+        "workload": CHUNKED, "value": world * flops / (ms["one"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "ms_per_call": ms["one"],
+        "roofline": roofline(flops / (ms["one"] * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s", "tensor",
+                             "prefill_kernel<128> + prefill_combine_kernel (events around segkv_prefill_attn)"),
+        "two_source": {"metric": "two-source chunked prefill TFLOP/s", "unit": "TFLOP/s",
+                       "value": world * flops / (ms["two"] * 1e-3) / 1e12, "ms_per_call": ms["two"],
+                       "ring_pages": {"two_source": r_two, "one_source": w.ring_pages},
+                       "local_ring_bytes_saved_per_sequence": n_local * (w.ring_pages - r_two) * page_bytes,
+                       "roofline": roofline(flops / (ms["two"] * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s",
+                                            "tensor", "prefill_kernel<128>, chunk pages from the call's K/V "
+                                                      "(events around segkv_prefill_attn_2src)")},
+        "append": {"bytes": app_b, "ms": t_app,
+                   "roofline": roofline(app_b / (t_app * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
+                                        "append_kernel (events around segkv_append of the 4096-token chunk)",
+                                        profiled_traffic("append_chunk128k.md", APPEND_SOURCES))},
+        "gpu_launches": 2 * min(args.steps, 20) * 2,
+    }
 
 
 def bench_fork(args, torch, dev, stream, max_over_ranks, world, pk):

@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kThreadsDec, 1)
     mbar_init(&bar->merge[0], 128);
     mbar_init(&bar->merge[1], 128);
     bar->abort_flag = 0;
+    set_wait_limit(p.g.wait_limit);
     fence_mbar_init();
     if (p.newk && blockIdx.x == 0) state[0] = p.cursor_after;
     pdl_launch_dependents();  // the combine kernel may start its CTAs; they wait for this grid

@@ -50,6 +50,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // stage, far below anything that would look like a hang.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
+// Cycle limit of the bounded waits of the running CTA: set once by thread 0 before the CTA's
+// first block-wide barrier (0 = kWaitLimitCycles).  A test may shorten it to make a wait run
+// out; the drain waits on the way out keep kWaitLimitCycles, so copies and MMAs in flight
+// always complete before a CTA exits.
+static __shared__ long long s_wait_limit;
+__device__ __forceinline__ void set_wait_limit(long long cycles) {
+  s_wait_limit = cycles > 0 ? cycles : kWaitLimitCycles;
+}
+
 // Bounded wait for the phase with the given parity.  Returns false (and raises the CTA's
 // abort flag and the device error word) when the limit passes or another role aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
@@ -61,7 +70,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > s_wait_limit) {
       *abort_flag = 1;
       set_error(state, kErrDeviceTimeout);
       return false;

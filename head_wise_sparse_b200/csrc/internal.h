@@ -61,6 +61,7 @@ struct StorageGeom {  // what every kernel needs to resolve a logical position t
   int32_t *state;
   void *k_pool, *v_pool;
   int num_pages, page, head_dim, hkv, hq, max_seqs, max_lp, ring, window;
+  long long wait_limit;  // cycle limit of the kernels' bounded waits (0: about two seconds)
 };
 
 // -- launchers (each .cu file exposes one host function per kernel) --------------------
@@ -104,6 +105,9 @@ struct PrefillLaunch {
   int store;
   const int32_t *pair_off;
   int cursor0, new_pages;
+  // Test hook: 1 makes the MMA thread first wait on a barrier nothing arrives on, so that its
+  // bounded wait runs out and every role takes the abort and drain path.
+  int stall_test;
 };
 // kcmap / vcmap: the two-source call's K/V tensors [tokens, hkv, D] (box 64 x 1 x page);
 // unused (any valid map) when two_src == 0.

@@ -26,11 +26,15 @@
 //               row; fp32 online softmax in the exp2 domain, O rescaled only when the row
 //               maximum grows by more than 2^8; P (bf16) overwrites its S columns in TMEM,
 //               each half of 64 keys signalled as soon as it is stored;
+//               each row counts the key columns its mask keeps (the visited pairs);
 //               the epilogue reads O_t out of TMEM (and frees it for the next item at once),
 //               normalises it and writes bf16 out through a 128-byte-swizzled shared-memory
-//               buffer and TMA tile stores (64 columns at a time; scattered per-thread row
-//               stores would flood the SM's L2 request path that the K/V loads share),
-//               plus fp32 lse and visited counts.
+//               buffer, each warp storing its own 32 rows by TMA tile stores (64 columns at a
+//               time; scattered per-thread row stores would flood the SM's L2 request path
+//               that the K/V loads share), plus fp32 lse and visited counts.
+// No warp waits at a barrier that another warp must reach after a bounded wait (the only
+// block-wide barriers are at the start and the end), so an abort in any role lets every
+// other role leave its loop.
 // The two query tiles' chains (S -> softmax -> PV -> next S) interleave on the tensor core:
 // while one tile's warpgroup runs its softmax, the other tile's MMAs run.
 #include "device_common.cuh"
@@ -44,12 +48,12 @@ constexpr int kBN = 128;        // keys of one key tile
 constexpr int kStages = 2;      // K and V ring depth
 constexpr int kThreads = 384;
 // Registers per thread: 168 at launch (65536 / 384 rounded down to a multiple of 8);
-// warpgroup 0 drops to 72 and the two softmax warpgroups rise to 216, which adds up to the
-// launch total: 128 x 72 + 256 x 216 = 384 x 168 (setmaxnreg.inc can only take registers
+// warpgroup 0 drops to 80 and the two softmax warpgroups rise to 208, which stays within the
+// launch total: 128 x 80 + 256 x 208 <= 384 x 168 (setmaxnreg.inc can only take registers
 // the block was launched with).
 constexpr int kRegsLaunch = (65536 / kThreads) / 8 * 8;
-constexpr int kRegsLow = 72, kRegsHigh = (kRegsLaunch * kThreads - 128 * kRegsLow) / 256 / 8 * 8;
-static_assert(kRegsHigh == 216 && 128 * kRegsLow + 256 * kRegsHigh <= kRegsLaunch * kThreads,
+constexpr int kRegsLow = 80, kRegsHigh = (kRegsLaunch * kThreads - 128 * kRegsLow) / 256 / 8 * 8;
+static_assert(kRegsHigh == 208 && 128 * kRegsLow + 256 * kRegsHigh <= kRegsLaunch * kThreads,
               "register split exceeds the launch total");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
 // One exponential pair in kEmuEvery may go to the FMA pipe (exp2_fma2) instead of the
@@ -85,7 +89,7 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_lo[2], p_hi[2], pv_done[2], o_free[2];
-  uint64_t mma_done;
+  uint64_t mma_done, never;  // never: no one arrives (the stall test waits on it)
   uint64_t sched_full[4], sched_empty[4];
   int sched[4];
   Item sched_item[4];  // the producer decodes each item once; consumers read it here
@@ -151,7 +155,10 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
   // every chunk page is stored exactly once; a stage is reloaded only after those stores
   // have read it.
   int i = 0, c = 0;
-  bool ok = true, q_loaded = false;
+  // loads of the current tile / item already issued (bit 0: K, bit 1: V, bit 2: Q): with c and
+  // i they say which loads the drain on the way out must wait for
+  int issued = 0;
+  bool ok = true;
   // next item index, fetched one item ahead so its Q rows can be pulled into L2 early
   auto fetch = [&]() -> int {
     int v = 0;
@@ -185,7 +192,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
           tma_load_3d(q_s + t * S::kQTileBytes + hh * kTileRows * 128, &qmap, &bar->q_full, hh * 64, it.h * G,
                       it.q_row + t * p.tile_pos);
     }
-    q_loaded = true;
+    issued |= 4;
     const long long row_base = (((long long)p.layer * p.g.max_seqs + it.seq_id) * p.g.hkv + it.h) * p.g.max_lp;
     const int last_lp = (it.kv_len - 1) / P;
     int lp_base = -(1 << 30), pid = p.g.num_pages;
@@ -223,6 +230,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
               tma_load_3d(dst, &kmap, &bar->k_full[s], hh * 64, 0, phys);
           }
       }
+      issued |= 1;
       if (!(ok = warp_wait(&bar->v_empty[s], (u & 1) ^ 1, abort_flag, state))) break;
       if (lane == 0) mbar_expect_tx(&bar->v_full[s], S::kTileBytes);
       for (int j = 0; j < PPT; ++j) {
@@ -236,6 +244,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
               tma_load_3d(dst, &vmap, &bar->v_full[s], hh * 64, 0, phys);
           }
       }
+      issued |= 2;
       if constexpr (STORE) {
         // lane j: page j of this tile, if this item stores it (its id, else -1)
         int sp = -1;
@@ -276,19 +285,22 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
         }
       }
       ++c;
+      issued &= 4;
     }
     if (!ok) break;
     ++i;
+    issued = 0;
     idx = next;
   }
-  // drain: no copy of this CTA may still be in flight when it exits
-  for (int k = c - 1; k >= 0 && k >= c - kStages; --k) {
-    const int s = k % kStages;
-    const uint32_t u = (uint32_t)(k / kStages);
-    mbar_wait_drain(&bar->k_full[s], u & 1);
-    mbar_wait_drain(&bar->v_full[s], u & 1);
-  }
-  if (q_loaded) mbar_wait_drain(&bar->q_full, (uint32_t)((ok ? i - 1 : i) & 1));
+  // drain: no copy of this CTA may still be in flight when it exits.  On a stage only the last
+  // load issued can still be in flight (each later load of a stage waited for the earlier one
+  // to be consumed), likewise for the Q buffer.
+  const int k_issued = c + (issued & 1), v_issued = c + ((issued >> 1) & 1), q_issued = i + ((issued >> 2) & 1);
+  for (int k = k_issued - 1; k >= 0 && k >= k_issued - kStages; --k)
+    mbar_wait_drain(&bar->k_full[k % kStages], (uint32_t)(k / kStages) & 1);
+  for (int k = v_issued - 1; k >= 0 && k >= v_issued - kStages; --k)
+    mbar_wait_drain(&bar->v_full[k % kStages], (uint32_t)(k / kStages) & 1);
+  if (q_issued > 0) mbar_wait_drain(&bar->q_full, (uint32_t)(q_issued - 1) & 1);
   if constexpr (STORE) {
     if (lane == 0) bulk_wait_all();  // the pool holds every stored page before the CTA exits
   }
@@ -310,7 +322,8 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
   const uint32_t k_lo = (smem_u32(k_s) >> 4) | (1u << 16);
   const uint32_t v_lo = (smem_u32(v_s) >> 4) | ((uint32_t)(kBN * 128 >> 4) << 16);
   int i = 0, c = 0;
-  bool ok = true;
+  // stall test: a wait that runs out before any MMA is issued (nothing arrives on `never`)
+  bool ok = !p.stall_test || mbar_wait(&bar->never, 0, abort_flag, state);
   // O_t += P_t(cc) V(cc); the first PV of an item overwrites O_t
   auto issue_pv = [&](int t, int cc, bool first, bool last) -> bool {
     const int s = cc % kStages;
@@ -341,7 +354,7 @@ __device__ __forceinline__ void mma_role(const PrefillLaunch &p, Bars *bar, cons
               desc(kb + (kk >> 2) * (kBN * 128 >> 4) + (kk & 3) * 2), kIdescQK, kk > 0 ? 1u : 0u);
     umma_commit(&bar->s_full[t]);
   };
-  for (;;) {
+  while (ok) {
     const int slot = i & 3;
     if (!(ok = mbar_wait(&bar->sched_full[slot], (i >> 2) & 1, abort_flag, state))) break;
     const int idx = bar->sched[slot];
@@ -388,6 +401,12 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
   const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
   const uint32_t t_s = t_lane + S::col_s(tq), t_o = t_lane + S::col_o(tq);
   const float sl2 = p.scale_log2;
+  // this warp's 32 rows of its warpgroup's staging buffer, and the first (head, position) of
+  // those rows in the tile: the output map's box is the 32 rows one warp stores (min(G, 32)
+  // heads x max(1, 32 / G) positions)
+  uint8_t *stg = o_stage + tq * Smem<D>::kOStageBytes + q4 * 32 * 128;
+  const int box_h = (q4 * 32) % G, box_p = (q4 * 32) / G, warp_last = (q4 * 32 + 31) / G;
+  bool stored = false;  // a TMA store of this warp may still be reading its staging rows
   int i = 0, c = 0;
   for (;;) {
     const int slot = i & 3;
@@ -404,6 +423,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
     const int pq = min(p_raw, it.q_last);  // rows past the sequence repeat its last query
     const int lo = it.global ? 0 : max(0, pq - p.g.window + 1);
     float m_used = -INFINITY, l = 0.f;
+    uint32_t cnt = 0;  // key columns this row's mask keeps
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       if (!(ok = warp_wait(&bar->s_full[tq], c & 1, abort_flag, state))) break;
@@ -416,12 +436,19 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
       const int k0 = (it.kt_lo + j) * kBN;
       // warp-uniform branch: only tiles that cut some row's window edge or diagonal mask
       if (__any_sync(0xffffffffu, k0 < lo || k0 + kBN - 1 > pq)) {
-        // keep columns a..b of this tile: one unsigned compare per element
+        // keep columns a..b of this tile: one unsigned compare per element, and count them
         const int a = lo - k0;
         const unsigned span = (unsigned)(pq - lo);
+        uint32_t kept = 0;
 #pragma unroll
-        for (int jj = 0; jj < kBN; ++jj)
-          if ((unsigned)(jj - a) > span) s[jj] = -INFINITY;
+        for (int jj = 0; jj < kBN; ++jj) {
+          const bool keep = (unsigned)(jj - a) <= span;
+          s[jj] = keep ? s[jj] : -INFINITY;
+          kept += keep ? 1u : 0u;
+        }
+        cnt += kept;
+      } else {
+        cnt += kBN;  // every column of the tile is visible to every row of this warp
       }
       float mx8[8];
 #pragma unroll
@@ -523,28 +550,29 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
       }
       tc_fence_before();
       mbar_arrive(&bar->o_free[tq]);  // O_t is read: the next item's first PV may overwrite it
-      if (it.q_first + (tq + 1) * p.tile_pos - 1 <= it.q_last) {
-        // a tile whose rows are all real queries goes out through TMA; the last tile of a
-        // sequence may run past it (those rows belong to the next sequence) and is stored
-        // row by row
-        uint8_t *stg = o_stage + tq * Smem<D>::kOStageBytes;
-        const bool leader = (threadIdx.x & 127) == 0;
+      if (it.q_first + tq * p.tile_pos + warp_last <= it.q_last) {
+        // the warp's 32 rows are all real queries: stored by TMA from this warp's staging rows;
+        // the last tile of a sequence may run past it (those rows belong to the next
+        // sequence) and is stored row by row
 #pragma unroll
         for (int hh = 0; hh < D / 64; ++hh) {
-          if (leader) bulk_wait_read_all();  // the previous store has read the buffer
-          named_bar_sync(1 + tq, 128);
-          // row r of the box at r * 128 bytes, 16-byte chunk c at (c ^ (r mod 8)): the
-          // 128-byte swizzle the output tensor map expects
+          if (stored) {
+            if (lane == 0) bulk_wait_read_all();  // the previous store has read these rows
+            __syncwarp();
+          }
+          // row r at r * 128 bytes, 16-byte chunk c at (c ^ (r mod 8)): the 128-byte swizzle
+          // the output tensor map expects
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4 *>(stg + row * 128 + ((c ^ (row & 7)) << 4)) =
+            *reinterpret_cast<uint4 *>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
                 make_uint4(w[hh * 32 + 4 * c], w[hh * 32 + 4 * c + 1], w[hh * 32 + 4 * c + 2], w[hh * 32 + 4 * c + 3]);
           fence_async_smem();
-          named_bar_sync(1 + tq, 128);
-          if (leader) {
-            tma_store_3d(&omap, stg, hh * 64, it.h * G, it.q_row + tq * p.tile_pos);
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&omap, stg, hh * 64, it.h * G + box_h, it.q_row + tq * p.tile_pos + box_p);
             bulk_commit();
           }
+          stored = true;
         }
       } else if (valid) {
         uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow * D);
@@ -554,19 +582,18 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
     }
     if (valid && it.slot < 0) p.lse[orow] = (m_used + fast_log2(l)) * 0.69314718055994531f;
     if (p.visited) {
-      // visible keys of this row inside the item's key tiles (all of them unless chunked)
-      const int k_lo = max(lo, it.kt_lo * kBN), k_hi = min(pq, it.kt_hi * kBN + kBN - 1);
-      unsigned long long cnt = (valid && k_hi >= k_lo) ? (unsigned long long)(k_hi - k_lo + 1) : 0ull;
+      // the key columns the row's mask kept in the item's key tiles (all of them unless chunked)
+      unsigned long long n = valid ? (unsigned long long)cnt : 0ull;
       if (G < 32) {
-        for (int off = G; off < 32; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-        if (lane < G && cnt) atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + lane], cnt);
-      } else if (cnt) {
-        atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + g], cnt);
+        for (int off = G; off < 32; off <<= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
+        if (lane < G && n) atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + lane], n);
+      } else if (n) {
+        atomicAdd(&p.visited[(long long)it.b * p.g.hq + it.h * G + g], n);
       }
     }
     ++i;
   }
-  if ((threadIdx.x & 127) == 0) bulk_wait_all();  // no store of this warpgroup outlives the CTA
+  if (lane == 0) bulk_wait_all();  // no store of this warp outlives the CTA
 }
 
 template <int D, bool TWO, bool STORE>
@@ -610,11 +637,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar->o_free[t], 128);
     }
     mbar_init(&bar->mma_done, 1);
+    mbar_init(&bar->never, 1);
     for (int s = 0; s < 4; ++s) {
       mbar_init(&bar->sched_full[s], 1);
       mbar_init(&bar->sched_empty[s], 9);  // MMA thread + lane 0 of each of the 8 softmax warps
     }
     bar->abort_flag = 0;
+    set_wait_limit(p.g.wait_limit);
     fence_mbar_init();
     if (STORE && blockIdx.x == 0) state[0] = p.cursor0 + p.new_pages;
   }

@@ -384,6 +384,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       mbar_init(&bar->sched_empty[s], 1 + kRReducers);  // MMA thread + lane 0 of each reducing warp
     }
     bar->abort_flag = 0;
+    set_wait_limit(p.g.wait_limit);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(&bar->tmem_base, kRSBufs * kRCols);

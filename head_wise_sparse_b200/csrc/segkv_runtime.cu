@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <random>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -90,6 +91,11 @@ struct segkv {
   CUtensorMap kmap, vmap;
   int num_sms = 0;
   std::string last_error;  // which CUDA step failed last, and why
+  // test hooks (segkv_debug_set): the kernels' wait limit in cycles (0: default), a one-shot
+  // stall of the next prefill launch, and the order in which a prefill call's work list runs
+  long long wait_limit = 0;
+  int stall_next_prefill = 0;
+  long long lpt_order = 0;
 };
 
 namespace {
@@ -120,6 +126,7 @@ StorageGeom geom(const segkv_t *h) {
   g.max_lp = h->max_lp;
   g.ring = h->ring;
   g.window = h->cfg.window;
+  g.wait_limit = h->wait_limit;
   return g;
 }
 
@@ -448,6 +455,10 @@ const char *segkv_strerror(int s) {
   }
 }
 
+namespace {
+int noalloc_scratch(segkv_t *h, void **ptr);
+}
+
 int segkv_create(const segkv_config *c, segkv_t **out) {
   if (!c || !out) return SEGKV_ERR_INVALID_ARG;
   *out = nullptr;
@@ -480,6 +491,20 @@ int segkv_create(const segkv_config *c, segkv_t **out) {
   h->ref.assign((size_t)c->num_pages, 0);
   h->ref_scratch.assign((size_t)c->num_pages, 0);
   h->cfg.head_class = nullptr;
+  // Set-up of the allocation-free decode: with a device current, look up (and so make
+  // resident) the library's fixed scratch array on it now, before the caller hands the rest
+  // of the device to its own allocator.  Without a device (a host-only process) there is
+  // nothing to set up.
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    void *scratch = nullptr;
+    if (noalloc_scratch(h, &scratch) != SEGKV_OK) {
+      delete h;
+      return SEGKV_ERR_CUDA;
+    }
+  } else {
+    cudaGetLastError();  // clear the sticky "no device" status of the runtime
+  }
   *out = h;
   return SEGKV_OK;
 }
@@ -496,6 +521,26 @@ void segkv_destroy(segkv_t *h) {
 
 int segkv_ring_pages(const segkv_t *h) { return h ? h->ring : -1; }
 const char *segkv_last_error(const segkv_t *h) { return h ? h->last_error.c_str() : "no handle"; }
+
+int segkv_debug_set(segkv_t *h, int key, long long value) {
+  if (!h) return SEGKV_ERR_INVALID_ARG;
+  switch (key) {
+    case SEGKV_DEBUG_WAIT_LIMIT:
+      if (value < 0) return SEGKV_ERR_INVALID_ARG;
+      h->wait_limit = value;
+      return SEGKV_OK;
+    case SEGKV_DEBUG_STALL_NEXT_PREFILL:
+      if (value != 0 && value != 1) return SEGKV_ERR_INVALID_ARG;
+      h->stall_next_prefill = (int)value;
+      return SEGKV_OK;
+    case SEGKV_DEBUG_PREFILL_ORDER:
+      if (value < 0) return SEGKV_ERR_INVALID_ARG;
+      h->lpt_order = value;
+      return SEGKV_OK;
+    default:
+      return SEGKV_ERR_INVALID_ARG;
+  }
+}
 int segkv_max_lp(const segkv_t *h) { return h ? h->max_lp : -1; }
 int segkv_pages_used(const segkv_t *h) { return h ? (int)h->pages_used : -1; }
 
@@ -808,6 +853,14 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
   std::vector<PlanChunk> chunks;
   std::vector<SplitGroup> groups;
   split_long_items(h, layer, q_start_pos, q_len, items, h->num_sms, chunks, groups);
+  if (h->lpt_order != 0) {  // test hook: run the same work list in another order
+    if (h->lpt_order == 1) {
+      std::reverse(chunks.begin(), chunks.end());
+    } else {
+      std::mt19937_64 rng((uint64_t)h->lpt_order);
+      std::shuffle(chunks.begin(), chunks.end(), rng);
+    }
+  }
   const int items_off = (int)align_up(kHeaderBytes + sizeof(PrefillSeq) * nseq, 16);
   const int groups_off = items_off + 16 * (int)chunks.size();
   const int pair_off_at = groups_off + 16 * (int)groups.size();
@@ -838,12 +891,14 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
     gr[i] = make_int4(g.b, (int)make_item_w1(h->cls[layer * H + g.h] != 0, g.h, g.t), g.first_slot, g.n);
   }
   if (!pair_off.empty()) std::memcpy(static_cast<char *>(host) + pair_off_at, pair_off.data(), 4 * pair_off.size());
-  CUtensorMap qmap, omap;  // query in, output out: the same [tokens, Hq, D] geometry and tile box
+  // query in (box: one 128-row tile, G heads x 128/G positions) and output out (box: the 32
+  // rows one softmax warp stores, min(G, 32) heads x max(1, 32/G) positions), both [tokens, Hq, D]
+  CUtensorMap qmap, omap;
   const int D = h->cfg.head_dim, Hq = h->cfg.num_q_heads, Hkv = h->cfg.num_kv_heads;
   if (!make_map(&qmap, q, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
                 kPrefillTileRows / h->G) ||
-      !make_map(&omap, out, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, h->G,
-                kPrefillTileRows / h->G)) {
+      !make_map(&omap, out, D, Hq, (uint64_t)tq, (uint64_t)D * 2, (uint64_t)Hq * D * 2, std::min(h->G, 32),
+                std::max(1, 32 / h->G))) {
     h->last_error = "query/output tensor map encode failed";
     return SEGKV_ERR_CUDA;
   }
@@ -877,6 +932,8 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.two_src = two ? 1 : 0;
+  p.stall_test = h->stall_next_prefill;
+  h->stall_next_prefill = 0;
   if (fused) {
     p.store = 1;
     p.pair_off = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + pair_off_at);
@@ -1180,7 +1237,10 @@ unsigned char g_noalloc_meta[kNoAllocMetaBytes];
 uint64_t g_noalloc_seen[kNoAllocMaxSeqSlots / 64];
 void *g_noalloc_dev_ptr[kNoAllocMaxDevices];
 
-// Device address of the scratch array on the current device, looked up once per device.
+// Device address of the scratch array on the current device, looked up once per device
+// (segkv_create does it for the device current there; a call on another device does it on
+// its first call there).  The look-up loads the module that holds the array, so this is where
+// its 64 MiB become resident on that device.
 int noalloc_scratch(segkv_t *h, void **ptr) {
   int dev = 0;
   SEGKV_CUDA(h, "cudaGetDevice", cudaGetDevice(&dev));

@@ -26,8 +26,11 @@ EXPORTS = [
     "segkv_workspace_bytes", "segkv_reset", "segkv_append", "segkv_prefill_attn", "segkv_plan_prefill",
     "segkv_decode_attn", "segkv_device_status", "segkv_strerror", "segkv_last_error",
     "segkv_decode_attn_noalloc", "segkv_relocate_q", "segkv_fork", "segkv_decode_step",
-    "segkv_router_topk", "segkv_prefill_attn_2src", "segkv_prefill_append",
+    "segkv_router_topk", "segkv_prefill_attn_2src", "segkv_prefill_append", "segkv_debug_set",
 ]
+
+# keys of segkv_debug_set (test hooks; see include/segkv.h)
+DEBUG_WAIT_LIMIT, DEBUG_STALL_NEXT_PREFILL, DEBUG_PREFILL_ORDER = 1, 2, 3
 
 
 class SegkvError(RuntimeError):
@@ -83,6 +86,7 @@ def lib():
         L.segkv_device_status.argtypes = [P, P]
         L.segkv_last_error.argtypes = [P]
         L.segkv_last_error.restype = ctypes.c_char_p
+        L.segkv_debug_set.argtypes = [P, I, ctypes.c_longlong]
         L.segkv_strerror.argtypes = [I]
         L.segkv_strerror.restype = ctypes.c_char_p
         _lib = L
@@ -241,6 +245,9 @@ class Handle:
     def device_status(self, stream=None) -> int:
         return lib().segkv_device_status(self.h, _stream(stream))
 
+    def debug_set(self, key: int, value: int) -> int:
+        return lib().segkv_debug_set(self.h, key, value)
+
 
 # ---------------------------------------------------------------------------- torch front end
 class SegKV:
@@ -371,3 +378,7 @@ class SegKV:
 
     def device_status(self) -> int:
         return self.handle.device_status()
+
+    def debug_set(self, key: int, value: int) -> None:
+        """segkv_debug_set (test hooks): the wait limit, a stalled prefill, the work-list order."""
+        _check(self.handle.debug_set(key, value), "segkv_debug_set", self.handle.h)

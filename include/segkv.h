@@ -279,12 +279,17 @@ int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
  *   until the process exits); per-call metadata is staged in a fixed 1 MiB host buffer.
  *   A call that would need more returns SEGKV_ERR_WORKSPACE and names the sizes in
  *   segkv_last_error.  Nothing is allocated: no cudaMalloc, cudaFree or cudaHostAlloc.
- *   The first call on a device looks up the array's device address (once per device);
- *   make that first call before any stream capture.
+ *   Set-up: segkv_create looks up the array's device address on the device current at
+ *   that moment, which makes the 64 MiB resident there; create the handle before handing
+ *   the rest of the device to another allocator.  A call on a device that no segkv_create
+ *   saw does the look-up itself (once per device); make that first call before any stream
+ *   capture.
  *   Every call shares the one array and the scheduler counter is re-zeroed by each call's
  *   metadata copy, so calls that overlap on the GPU (different streams, or different
  *   handles) race and give wrong results: issue them one after another on one stream.
- *   Not thread-safe.
+ *   The host metadata buffer and the duplicate-id check's bitmap are shared by every
+ *   handle of the process as well: calls from different host threads race there too, even
+ *   on different handles.  Not thread-safe.
  */
 int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,
                               const void *q, float softmax_scale, int num_splits, void *out, float *lse,
@@ -320,6 +325,27 @@ const char *segkv_last_error(const segkv_t *h);
 
 /* Static description of a status code. */
 const char *segkv_strerror(int status);
+
+/* Test hooks.  The pages describe no such control; these exist so that the failure paths
+ * and the scheduler's order independence can be exercised without faulting a GPU.
+ *   SEGKV_DEBUG_WAIT_LIMIT: cycle limit of the bounded pipeline waits of every later launch
+ *     of this handle (value >= 0; 0 restores the default of about two seconds).  A wait that
+ *     runs out sets SEGKV_ERR_DEVICE_TIMEOUT in the error word; the kernel then lets its
+ *     copies and MMAs in flight finish, frees its tensor memory and returns.
+ *   SEGKV_DEBUG_STALL_NEXT_PREFILL: value 1 makes the next prefill launch of this handle wait
+ *     first on a barrier that nothing arrives on, so that the wait runs out (one shot; the
+ *     call's outputs are then undefined and segkv_device_status reports the timeout).
+ *   SEGKV_DEBUG_PREFILL_ORDER: 0 runs a prefill call's work list longest first (the
+ *     default); 1 runs it in reverse; any other value shuffles it with that seed.  Every item
+ *     is computed by one CTA in a fixed key order, so outputs do not depend on it.
+ * Returns INVALID_ARG for a null handle, an unknown key or a value out of range.  Not
+ * thread-safe, like every call on a handle. */
+enum {
+  SEGKV_DEBUG_WAIT_LIMIT = 1,
+  SEGKV_DEBUG_STALL_NEXT_PREFILL = 2,
+  SEGKV_DEBUG_PREFILL_ORDER = 3
+};
+int segkv_debug_set(segkv_t *h, int key, long long value);
 
 #ifdef __cplusplus
 }

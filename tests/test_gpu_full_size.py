@@ -1,5 +1,8 @@
 """Full-size workloads on the CUDA path (needs a B200), in the launch configuration the
-benchmark times, checked on sampled rows the oracle computes one by one, plus edge cases.
+benchmark times, plus edge cases.  The Mistral-shaped and 128K-chunk workloads are checked
+on every (token, head) row against the oracle (seconds to about a minute of fp64 on the
+host's cores); the Llama-shaped 4-layer workload (about 34 TFLOP in fp64) on sampled rows
+the oracle computes one by one.
 
 Tolerances as in test_gpu_parity: |out - ref| <= 8e-3 + 1e-2 |ref|, |lse - ref| <= 1e-3;
 page tables and visited-pair counts bit-exact (counts against the closed forms in
@@ -84,10 +87,15 @@ def prefill_full(torch, w, layer_list, n_rows, ctx_chunk=4096, golden=None):
         out, lse = kv.prefill(layer, ids, qs, ql, to_dev(q), visited=vis)
         torch.cuda.synchronize()
         assert kv.device_status() == 0
-        rows = sample_rows(w, ql, n_rows, seed=layer)
-        ro, rl, _ = o.attention(layer, ids, qs, ql, q, rows=rows)
-        compare_rows(w, out, lse, ro, rl, rows)
         got = vis.cpu().numpy().astype(np.uint64)
+        if n_rows is None:  # every row, and the oracle's own visited counts
+            ro, rl, rc = o.attention(layer, ids, qs, ql, q)
+            compare_rows(w, out, lse, ro, rl, np.arange(ro.reshape(-1, w.d).shape[0]))
+            assert np.array_equal(got, rc)
+        else:
+            rows = sample_rows(w, ql, n_rows, seed=layer)
+            ro, rl, _ = o.attention(layer, ids, qs, ql, q, rows=rows)
+            compare_rows(w, out, lse, ro, rl, rows)
         assert np.array_equal(got, closed_form_counts(w, layer, ids, qs, ql))
         if golden:
             g = json.load(open(os.path.join(GOLDEN, "visible_pairs.json")))[golden]
@@ -98,12 +106,12 @@ def prefill_full(torch, w, layer_list, n_rows, ctx_chunk=4096, golden=None):
     return kv
 
 
-def test_mistral7b_prefill_full_size(torch_cuda):
-    prefill_full(torch_cuda, wl.CONFIGS["mistral7b_prefill_L8192"], [0], 3000, golden="mistral7b_prefill_L8192")
+def test_mistral7b_prefill_full_size_every_row(torch_cuda):
+    prefill_full(torch_cuda, wl.CONFIGS["mistral7b_prefill_L8192"], [0], None, golden="mistral7b_prefill_L8192")
 
 
-def test_chunked_128k_prefill_full_size(torch_cuda):
-    prefill_full(torch_cuda, wl.CONFIGS["mha_chunked_prefill_128k"], [0], 2000, golden="mha_chunked_prefill_128k")
+def test_chunked_128k_prefill_full_size_every_row(torch_cuda):
+    prefill_full(torch_cuda, wl.CONFIGS["mha_chunked_prefill_128k"], [0], None, golden="mha_chunked_prefill_128k")
 
 
 def test_llama70b_varlen_four_layers_full_size(torch_cuda):

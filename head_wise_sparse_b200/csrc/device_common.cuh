@@ -267,28 +267,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^x for a pair of lanes on the FMA pipe, to take part of the exponentials off the MUFU.
-// Cody-Waite style split x = j + f with j = round(x) and f in [-1/2, 1/2]; 2^f by a
-// degree-3 polynomial whose coefficients minimise the relative error on that interval
-// (fitted by exp2_poly_fit.py beside this file; max relative error 7.5e-5 in fp32, far
-// below bf16's 2^-9); 2^j is added to the exponent field.  x is clamped at -125 so the
-// result stays a normal number: x = -inf gives about 2.4e-38 instead of 0, negligible
-// against a row sum that is at least 1.
-constexpr float kExp2C0 = 0.99992805719f, kExp2C1 = 0.69326096773f, kExp2C2 = 0.24261112511f,
-                kExp2C3 = 0.05517166480f;
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));  // 1.5 * 2^23: round to integer
-  const float2 j = fadd2(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = ffma2(j, make_float2(-1.f, -1.f), x);
-  float2 q = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-  q = ffma2(q, f, make_float2(kExp2C1, kExp2C1));
-  q = ffma2(q, f, make_float2(kExp2C0, kExp2C0));
-  // the low mantissa bits of t hold j; the bits above them shift out with << 23
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
-}
 __device__ __forceinline__ float fast_log2(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -68,10 +68,11 @@ struct StorageGeom {  // what every kernel needs to resolve a logical position t
 cudaError_t launch_reset(const StorageGeom &g, int num_layers, cudaStream_t st);
 
 // Copies on write first (n_jobs > 0: jobs_dev[j] = (k_new, k_old, rows)), then the scatter;
-// plan_dev == NULL when no page of the call is shared.
+// plan_dev == NULL when no page of the call is shared; max_pages = the most pages the call
+// touches for one (sequence, head).
 cudaError_t launch_append(const StorageGeom &g, int layer, const void *ws_meta, int nseq, const uint8_t *cls_dev,
                           const int32_t *pair_off_dev, const int32_t *plan_dev, const int4 *jobs_dev, int n_jobs,
-                          int cursor0, int new_pages, int total_tokens, const void *k_new, const void *v_new,
+                          int cursor0, int new_pages, int max_pages, const void *k_new, const void *v_new,
                           cudaStream_t st);
 
 // A prefill work item is four int32 words: w0 = sequence index in the call, w1 as above

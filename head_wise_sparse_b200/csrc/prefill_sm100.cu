@@ -56,11 +56,6 @@ constexpr int kRegsLow = 80, kRegsHigh = (kRegsLaunch * kThreads - 128 * kRegsLo
 static_assert(kRegsHigh == 208 && 128 * kRegsLow + 256 * kRegsHigh <= kRegsLaunch * kThreads,
               "register split exceeds the launch total");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
-// One exponential pair in kEmuEvery may go to the FMA pipe (exp2_fma2) instead of the
-// MUFU; 0 keeps all of them on the MUFU.  Measured on the Mistral-shaped and 128K-chunk
-// workloads, every ratio from 1/8 to 1/2 was slower: the softmax here is bound by its
-// instruction stream and latency, not by MUFU throughput.
-constexpr int kEmuEvery = 0;
 
 template <int D>
 struct Smem {
@@ -489,11 +484,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap &omap, const Pref
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 x = ffma2(make_float2(s[qq * 32 + 2 * e], s[qq * 32 + 2 * e + 1]), c2, nm2);
-          float2 pe;
-          if (kEmuEvery > 0 && e % (kEmuEvery > 0 ? kEmuEvery : 1) == kEmuEvery - 1)
-            pe = exp2_fma2(x);
-          else
-            pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
           acc[e & 3] = fadd2(acc[e & 3], pe);
           pk[e] = pack_bf16x2(pe.x, pe.y);
         }

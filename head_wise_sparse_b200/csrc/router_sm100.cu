@@ -296,8 +296,8 @@ __device__ __forceinline__ void router_reduce(const RouterLaunch &p, RBars *bar,
       float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
       tmem_ld_wait();
       if (full) {
-        // (moving a quarter of these exponentials to the FMA pipe with exp2_fma2 measured
-        // 2 % slower: the loop is bound by issue and latency, not by the MUFU)
+        // (moving a quarter of these exponentials to an FMA-pipe polynomial measured 2 %
+        // slower: the loop is bound by issue and latency, not by the MUFU)
 #pragma unroll
         for (int c = 0; c < kHalf; c += 4) {
           const float4 l = nl[c / 4];

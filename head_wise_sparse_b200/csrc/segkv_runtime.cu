@@ -660,6 +660,7 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
   } scratch_clear{h->ref_scratch, ref_keys};
   auto ref_of = [&](int32_t k) { return h->ref[k] + h->ref_scratch[k]; };
   long long new_pages = 0;
+  int max_pages = 0;  // the most pages one (sequence, head) of the call touches
   for (int b = 0; b < nseq; ++b)
     for (int k = 0; k < H; ++k) {
       pair_page[(size_t)b * H + k] = (int32_t)plan.size();
@@ -669,6 +670,7 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
       size_t row;
       bool global;
       touched(b, k, lp0, lp1, row, global);
+      max_pages = std::max(max_pages, lp1 - lp0 + 1);
       if (!copies) {  // a page is taken exactly for an empty slot
         for (int lp = lp0; lp <= lp1; ++lp) new_pages += h->slot_k[row + (global ? lp : lp % R)] < 0;
         continue;
@@ -724,7 +726,7 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
   const int4 *jobs_dev = reinterpret_cast<const int4 *>(static_cast<const char *>(ws) + jobs_off);
   SEGKV_CUDA(h, "append launch",
              launch_append(geom(h), layer, ws, nseq, cls_dev, off_dev, copies ? plan_dev : nullptr, jobs_dev,
-                           (int)jobs.size(), (int)h->pages_used, (int)new_pages, (int)total, k_new, v_new, st));
+                           (int)jobs.size(), (int)h->pages_used, (int)new_pages, max_pages, k_new, v_new, st));
   if (copies) {
     for (const auto &e : slot_set) {
       h->slot_k[e.first] = e.second;

@@ -574,6 +574,41 @@ def bench_tiny(args, torch, dev, stream, max_over_ranks, world, pk):
             "gpu_launches": len(ev)}
 
 
+def bench_append_layer(args, torch, dev, stream, max_over_ranks, world, pk):
+    """The append of one Llama-shaped layer (4 sequences of the seeded lengths, Hkv 8, D 128,
+    181 MB of K/V read and written) into an emptied handle, alone (the profiling leg)."""
+    w = wl.CONFIGS[HEADLINE].scaled(layers=1, classes=wl.CONFIGS[HEADLINE].classes[:1])
+    lens = [s.length for s in w.seqs]
+    ids, T = list(range(len(lens))), int(sum(lens))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(13)
+    k = torch.randn((T, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    v = torch.randn((T, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    kv = new_handle(w, dev, ws_tokens=T, max_chunk=max(lens))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    times = []
+    for i in range(args.warmup + args.steps):
+        kv.handle.reset(stream)
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kv.append(0, ids, [0] * len(lens), lens, k, v)
+        e1.record(stream)
+        if i >= args.warmup:
+            times.append((e0, e1))
+    torch.cuda.synchronize()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the append leg")
+    t = max_over_ranks(sum(a.elapsed_time(b) for a, b in times) / len(times))
+    b = append_bytes(w, T)
+    del kv, k, v, flush
+    torch.cuda.empty_cache()
+    return {"workload": "llama70b_one_layer_append", "bytes": b, "ms": t,
+            "roofline": roofline(b / (t * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
+                                 "append_kernel (events around segkv_append)",
+                                 profiled_traffic("append_llama70b_layer.md", APPEND_SOURCES))}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -582,7 +617,10 @@ def main():
     ap.add_argument("--impl", default="segkv", choices=["segkv", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--headline-only", action="store_true", help="only the headline workload (for profiling)")
+    ap.add_argument("--only", default="", choices=["", "headline", "mistral", "chunked", "tiny", "fork", "decode",
+                                                   "append"],
+                    help="run one leg alone (for profiling): the headline step, or one sub-workload; 'append' is the "
+                         "append of one Llama-shaped layer (181 MB of K/V, about 1 GB on the device)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -606,6 +644,20 @@ def main():
     sampler = ClockSampler(str(getattr(props, "uuid", "")))
     time.sleep(0.3)
 
+    if args.only and args.only != "headline":
+        legs = {"mistral": lambda: bench_mistral(args, torch, dev, stream, max_over_ranks, world, pk),
+                "chunked": lambda: bench_chunked(args, torch, dev, stream, max_over_ranks, world, pk),
+                "tiny": lambda: bench_tiny(args, torch, dev, stream, max_over_ranks, world, pk),
+                "fork": lambda: bench_fork(args, torch, dev, stream, max_over_ranks, world, pk),
+                "decode": lambda: bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk),
+                "append": lambda: bench_append_layer(args, torch, dev, stream, max_over_ranks, world, pk)}
+        res = legs[args.only]()
+        sampler.stop()
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"only": args.only, **res}), flush=True)
+        return 0
     head = bench_headline(args, torch, dev, stream, barrier, max_over_ranks, world, pk, sampler)
     t0, t1 = head.pop("clock_window")
     clocks = sampler.summary(t0, t1)
@@ -618,7 +670,7 @@ def main():
         "peaks": {"source": pk_src, **pk},
     }
     appends = {"llama70b_4_layers": head["append"]}
-    if not args.headline_only:
+    if not args.only:
         mis = bench_mistral(args, torch, dev, stream, max_over_ranks, world, pk)
         appends["mistral7b"] = mis.pop("append")
         line["relocate"] = mis.pop("relocate")

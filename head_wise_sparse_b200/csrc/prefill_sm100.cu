@@ -145,14 +145,40 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
   // it): a page of the call's own query range comes from the caller's K/V tensors, packed
   // like q; only the context before the range is read from the pages.  Such a page's lane
   // holds -1 - (its first row in those tensors) instead of a page id.
-  // Fused append (STORE): once such a page has landed in shared memory, the item whose query
-  // range holds the page's first position also writes it to its pool page by TMA store, so
-  // every chunk page is stored exactly once; a stage is reloaded only after those stores
-  // have read it.
+  // Fused append (STORE): the item whose query range holds a chunk page's first position also
+  // writes that page from shared memory to its pool page by TMA store, so every chunk page is
+  // stored exactly once.  A tile's pages are stored one tile late, after the next tile's loads
+  // are issued (by then they have landed, so the producer does not wait for its own loads),
+  // with the pool ids worked out while the tile's own item was current; the last tile is
+  // stored after the loop.  A stage is reloaded only after the stores that read it have read
+  // it (bulk_wait_read_all before each K load).
   int i = 0, c = 0;
   // loads of the current tile / item already issued (bit 0: K, bit 1: V, bit 2: Q): with c and
   // i they say which loads the drain on the way out must wait for
   int issued = 0;
+  int sp_prev = -1, c_prev = -1;  // STORE: lane j = pool id of page j of tile c_prev to store, else -1
+  // STORE: writes the chunk pages of tile cs (lane j: page j's pool id in sp, else -1)
+  auto store_tile = [&](int sp, int cs) -> bool {
+    if (cs < 0 || !__ballot_sync(0xffffffffu, sp >= 0)) return true;
+    const int st = cs % kStages;
+    const uint32_t us = (uint32_t)(cs / kStages);
+    if (!warp_wait(&bar->k_full[st], us & 1, abort_flag, state)) return false;
+    for (int j = 0; j < PPT; ++j) {
+      const int ph = __shfl_sync(0xffffffffu, sp, j);
+      if (lane == 0 && ph >= 0)
+        for (int hh = 0; hh < S::kHalves; ++hh)
+          tma_store_3d(&kmap, k_s + st * S::kTileBytes + hh * kBN * 128 + j * P * 128, hh * 64, 0, ph);
+    }
+    if (!warp_wait(&bar->v_full[st], us & 1, abort_flag, state)) return false;
+    for (int j = 0; j < PPT; ++j) {
+      const int ph = __shfl_sync(0xffffffffu, sp, j);
+      if (lane == 0 && ph >= 0)
+        for (int hh = 0; hh < S::kHalves; ++hh)
+          tma_store_3d(&vmap, v_s + st * S::kTileBytes + hh * kBN * 128 + j * P * 128, hh * 64, 0, ph);
+    }
+    if (lane == 0) bulk_commit();
+    return true;
+  };
   bool ok = true;
   // next item index, fetched one item ahead so its Q rows can be pulled into L2 early
   auto fetch = [&]() -> int {
@@ -241,6 +267,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
       }
       issued |= 2;
       if constexpr (STORE) {
+        if (!(ok = store_tile(sp_prev, c_prev))) break;  // the previous tile's pages
         // lane j: page j of this tile, if this item stores it (its id, else -1)
         int sp = -1;
         if (lane < PPT) {
@@ -261,23 +288,8 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
             }
           }
         }
-        if (__ballot_sync(0xffffffffu, sp >= 0)) {
-          if (!(ok = warp_wait(&bar->k_full[s], u & 1, abort_flag, state))) break;
-          for (int j = 0; j < PPT; ++j) {
-            const int ph = __shfl_sync(0xffffffffu, sp, j);
-            if (lane == 0 && ph >= 0)
-              for (int hh = 0; hh < S::kHalves; ++hh)
-                tma_store_3d(&kmap, k_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, hh * 64, 0, ph);
-          }
-          if (!(ok = warp_wait(&bar->v_full[s], u & 1, abort_flag, state))) break;
-          for (int j = 0; j < PPT; ++j) {
-            const int ph = __shfl_sync(0xffffffffu, sp, j);
-            if (lane == 0 && ph >= 0)
-              for (int hh = 0; hh < S::kHalves; ++hh)
-                tma_store_3d(&vmap, v_s + s * S::kTileBytes + hh * kBN * 128 + j * P * 128, hh * 64, 0, ph);
-          }
-          if (lane == 0) bulk_commit();
-        }
+        sp_prev = sp;
+        c_prev = c;
       }
       ++c;
       issued &= 4;
@@ -286,6 +298,9 @@ __device__ __forceinline__ void producer_role(const CUtensorMap &qmap, const CUt
     ++i;
     issued = 0;
     idx = next;
+  }
+  if constexpr (STORE) {
+    if (ok) store_tile(sp_prev, c_prev);  // the last tile's pages
   }
   // drain: no copy of this CTA may still be in flight when it exits.  On a stage only the last
   // load issued can still be in flight (each later load of a stage waited for the earlier one

@@ -359,6 +359,33 @@ def bench_headline(args, torch, dev, stream, barrier, max_over_ranks, world, pk,
     achieved = flops / (t_pre * 1e-3) / 1e12
     app_b = L * append_bytes(w, T)
 
+    # ------------------------------------------------------------------ query relocation
+    # one layer's queries a call (1.4 GB read, 1.4 GB written: no call finds its operands in
+    # L2), each layer's in turn with that layer's head classes, seeded offsets in [0, 2^20);
+    # calls back to back after a sleep kernel lets the host queue them ahead of the GPU
+    shift = torch.randint(0, 1 << 20, (T,), generator=gen, device=dev, dtype=torch.int32)
+    for l in range(L):
+        kv.relocate_q(l, q[l], shift, out=out[l])
+    n_rel = max(args.steps, 12)
+    evr = events(torch, n_rel, 2)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(4_000_000)
+    for i, e in enumerate(evr):
+        e[0].record(stream)
+        kv.relocate_q(i % L, q[i % L], shift, out=out[i % L])
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the relocation calls")
+    t_rel = max_over_ranks(mean_ms(evr, 0, 1))
+    rel_b = 2 * q[0].numel() * 2
+    relocate = {"metric": "query relocation GB/s", "value": world * rel_b / (t_rel * 1e-3) / 1e9, "unit": "GB/s",
+                "ms_per_call": t_rel, "bytes_per_call": rel_b, "calls": n_rel,
+                "queries": f"{T} tokens x {w.hq} heads x {w.d} (one layer of {HEADLINE})",
+                "l2": "operands of 2.8 GB a call, calls back to back",
+                "roofline": roofline(rel_b / (t_rel * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
+                                     "relocate_q_kernel (events around each segkv_relocate_q)")}
+
     # ------------------------------------------------------------------ end to end, host buffers
     # every step copies all 4 layers' Q, K and V in from pinned host memory and every layer's
     # output and lse back out
@@ -393,6 +420,7 @@ def bench_headline(args, torch, dev, stream, barrier, max_over_ranks, world, pk,
     res = {
         "value": world * flops / (t_step * 1e-3) / 1e12, "ms_per_step": t_step, "prefill_kernel_ms": t_pre,
         "append_ms": t_app, "flops_per_step": flops, "visible_pairs_per_layer": pairs, "e2e": e2e,
+        "relocate": relocate,
         "roofline": roofline(achieved, pk["bf16_tflops"], "TFLOP/s", "tensor",
                              "prefill_kernel<128> (events around the 4 segkv_prefill_attn calls of a step)",
                              profiled_traffic("prefill_llama70b_varlen.md", PREFILL_SOURCES),
@@ -490,24 +518,32 @@ def bench_mistral(args, torch, dev, stream, max_over_ranks, world, pk):
         "gpu_launches": 3 * args.steps,
     }
     # query relocation: local heads turned by -delta, the global head copied (one read + one
-    # write of every query element)
-    q_rel = torch.empty_like(q_d)
+    # write of every query element).  Calls run back to back, as a serving loop issues them,
+    # over three (input, output) pairs in turn: 402 MB, so no call finds its operands in L2,
+    # and each call writes back the lines the call before it left dirty, as a copy in steady
+    # state does.  A sleep kernel first lets the host queue the calls ahead of the GPU, so the
+    # events time the GPU's work, not the host's call overhead.
+    sets = [(q_d if i == 0 else q_d.clone(), torch.empty_like(q_d)) for i in range(3)]
     shift = torch.full((L,), 100000, dtype=torch.int32, device=dev)
-    for _ in range(args.warmup):
-        kv.relocate_q(0, q_d, shift, out=q_rel)
-    evr = events(torch, min(args.steps, 50), 2)
-    for e in evr:
-        flush.fill_(1)
+    for i in range(max(args.warmup, 3)):
+        kv.relocate_q(0, sets[i % 3][0], shift, out=sets[i % 3][1])
+    n_rel = max(args.steps, 30)
+    evr = events(torch, n_rel, 2)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(4_000_000)
+    for i, e in enumerate(evr):
         e[0].record(stream)
-        kv.relocate_q(0, q_d, shift, out=q_rel)
+        kv.relocate_q(0, sets[i % 3][0], shift, out=sets[i % 3][1])
         e[1].record(stream)
     torch.cuda.synchronize()
     t_rel = max_over_ranks(mean_ms(evr, 0, 1))
     rel_b = 2 * q_d.numel() * 2
     res["relocate"] = {"metric": "query relocation GB/s", "value": world * rel_b / (t_rel * 1e-3) / 1e9,
-                       "unit": "GB/s", "ms_per_call": t_rel, "bytes_per_call": rel_b,
+                       "unit": "GB/s", "ms_per_call": t_rel, "bytes_per_call": rel_b, "calls": n_rel,
+                       "l2": "three operand sets in turn (402 MB), calls back to back",
                        "roofline": roofline(rel_b / (t_rel * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
-                                            "relocate_q_kernel (events around segkv_relocate_q)")}
+                                            "relocate_q_kernel (events around each segkv_relocate_q)")}
+    del sets
     # attention as a router: every token's received attention mass and the top quarter
     k_top = [L // 4]
     rt_scores = torch.empty((L,), dtype=torch.float32, device=dev)
@@ -537,7 +573,7 @@ def bench_mistral(args, torch, dev, stream, max_over_ranks, world, pk):
                                           peak_source=f"MUFU ex2: 16 per clock per SM x {sms} SMs x 1965 MHz "
                                                       "(the maximum SM clock)"),
                      "gpu_launches": 3 * len(evt)}
-    del kv, flush, q_rel
+    del kv, flush
     torch.cuda.empty_cache()
     return res
 
@@ -670,10 +706,11 @@ def main():
         "peaks": {"source": pk_src, **pk},
     }
     appends = {"llama70b_4_layers": head["append"]}
+    line["relocate"] = head["relocate"]
     if not args.only:
         mis = bench_mistral(args, torch, dev, stream, max_over_ranks, world, pk)
         appends["mistral7b"] = mis.pop("append")
-        line["relocate"] = mis.pop("relocate")
+        line["relocate"]["mistral7b_8192"] = mis.pop("relocate")
         line["router"] = mis.pop("router")
         line["fused_append_prefill"] = mis.pop("fused_append_prefill")
         line["mistral7b"] = mis

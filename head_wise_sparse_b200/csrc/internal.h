@@ -174,8 +174,8 @@ struct RelocateLaunch {
   const void *q_in;
   void *q_out;
   int hq, hkv, head_dim, interleaved;
-  double log2_base;
-  uint32_t cls_bits[32];  // class of KV heads 0..1023: bit set = global (passes unchanged)
+  double theta[64];       // theta_i = base^(-2i/D) for i < D/2, in fp64
+  uint32_t cls_bits[32];  // class of QUERY heads 0..1023 (their KV head's): bit set = global (passes unchanged)
 };
 cudaError_t launch_relocate_q(const RelocateLaunch &p, int n_tokens, cudaStream_t st);
 

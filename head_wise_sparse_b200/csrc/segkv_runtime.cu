@@ -1193,8 +1193,8 @@ int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, 
   if (n_tokens == 0) return SEGKV_OK;
   if (!shift || !q_in || !q_out || !aligned(shift, 4) || !aligned(q_in, 16) || !aligned(q_out, 16))
     return SEGKV_ERR_INVALID_ARG;
-  const int H = h->cfg.num_kv_heads;
-  if (H > 1024 || n_tokens > (1 << 30)) return SEGKV_ERR_UNSUPPORTED;
+  const int H = h->cfg.num_kv_heads, Hq = h->cfg.num_q_heads;
+  if (Hq > 1024 || n_tokens > (1 << 30)) return SEGKV_ERR_UNSUPPORTED;
   RelocateLaunch p{};
   p.shift = shift;
   p.q_in = q_in;
@@ -1203,10 +1203,11 @@ int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, 
   p.hkv = H;
   p.head_dim = h->cfg.head_dim;
   p.interleaved = interleaved;
-  p.log2_base = std::log2((double)theta_base);
+  const double log2_base = std::log2((double)theta_base);
+  for (int i = 0; i < p.head_dim / 2; ++i) p.theta[i] = std::exp2(-2.0 * i / p.head_dim * log2_base);
   std::memset(p.cls_bits, 0, sizeof(p.cls_bits));
-  for (int k = 0; k < H; ++k)
-    if (h->cls[(size_t)layer * H + k]) p.cls_bits[k >> 5] |= 1u << (k & 31);
+  for (int q = 0; q < Hq; ++q)
+    if (h->cls[(size_t)layer * H + q / (Hq / H)]) p.cls_bits[q >> 5] |= 1u << (q & 31);
   SEGKV_CUDA(h, "relocate launch", launch_relocate_q(p, n_tokens, static_cast<cudaStream_t>(stream)));
   return SEGKV_OK;
 }

@@ -310,7 +310,7 @@ int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const int32_t *se
  *   shift: DEVICE int32 [n_tokens].  Angles are formed and reduced modulo 2 pi in fp64,
  *   the rotation is done in fp32 and rounded to bf16 (nearest even).
  * Errors: INVALID_ARG (pointers, alignment, theta_base <= 1, interleaved not 0/1),
- * UNSUPPORTED (more than 1024 KV heads), CUDA.
+ * UNSUPPORTED (more than 1024 query heads), CUDA.
  */
 int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, const void *q_in, void *q_out,
                      float theta_base, int interleaved, void *stream);

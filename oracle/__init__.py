@@ -150,13 +150,17 @@ class Oracle:
                   q: np.ndarray, scale: Optional[float] = None, rows: Optional[np.ndarray] = None,
                   threads: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
         """Returns (out fp64 [T, hq, d], lse fp64 [T, hq], counts u64 [nseq, hq]).  With ``rows``
-        (packed token * hq + q head) only those rows are computed; other entries are NaN."""
+        (packed token * hq + q head) only those rows are computed and written; the other
+        entries are NaN, except in outputs above 2^25 elements, where they are left unwritten
+        (undefined) so that sampling a few rows of a large call does not cost a fill of the
+        whole output."""
         s, qs, ql = _i32(seq_ids), _i32(q_start), _i32(q_len)
         qq = np.ascontiguousarray(q, dtype=np.uint16)
         T = int(ql.sum())
         assert qq.size == T * self.hq * self.d
-        out = np.full((T, self.hq, self.d), np.nan)
-        lse = np.full((T, self.hq), np.nan)
+        fill = rows is not None and T * self.hq * self.d <= (1 << 25)
+        out = np.full((T, self.hq, self.d), np.nan) if fill else np.empty((T, self.hq, self.d))
+        lse = np.full((T, self.hq), np.nan) if fill else np.empty((T, self.hq))
         counts = np.zeros((len(s), self.hq), dtype=np.uint64)
         rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
         sc = float(scale) if scale is not None else 1.0 / np.sqrt(self.d)

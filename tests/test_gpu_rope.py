@@ -30,15 +30,18 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
     return wl.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
 
 
-@pytest.mark.parametrize("d,interleaved,inplace", [(128, False, False), (128, True, True), (64, False, True),
-                                                   (64, True, False)])
-def test_relocation_matches_oracle(torch_cuda, d, interleaved, inplace):
+# hq 8: several tokens a CTA with a ragged last block (8 tokens a block at D 128, 16 at D 64);
+# hq 64 at D 128: one token a block; hq 128 at D 128: two passes of 512 16-byte units a token
+@pytest.mark.parametrize("d,interleaved,inplace,hkv,g", [(128, False, False, 4, 2), (128, True, True, 4, 2),
+                                                         (64, False, True, 4, 2), (64, True, False, 4, 2),
+                                                         (128, False, False, 8, 8), (128, True, True, 16, 8)])
+def test_relocation_matches_oracle(torch_cuda, d, interleaved, inplace, hkv, g):
     torch = torch_cuda
-    hkv, g = 4, 2
-    w = Workload(400 + d, "rope", 1, hkv * g, hkv, d, 64, 256, 8, (Seq(0, 64, 0, 64),), ((1, 0, 0, 1),))
+    cls = tuple(int(k % 3 == 0) for k in range(hkv))  # globals among locals, first head global
+    w = Workload(400 + d, "rope", 1, hkv * g, hkv, d, 64, 256, 8, (Seq(0, 64, 0, 64),), (cls,))
     kv = make_kv(w)
-    rng = np.random.default_rng([41, d, int(interleaved)])
-    T = 777
+    rng = np.random.default_rng([41, d, int(interleaved), hkv])
+    T = 777 if hkv * g <= 8 else 131
     q_bits = bf16_bits(rng.standard_normal((T, w.hq, d)))
     shift = rng.integers(-500000, 500000, size=T).astype(np.int32)
     q = to_dev(q_bits)

@@ -51,6 +51,7 @@ PREFILL_SOURCES = ["head_wise_sparse_b200/csrc/prefill_sm100.cu", "head_wise_spa
 DECODE_SOURCES = ["head_wise_sparse_b200/csrc/decode.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 ROUTER_SOURCES = ["head_wise_sparse_b200/csrc/router_sm100.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 APPEND_SOURCES = ["head_wise_sparse_b200/csrc/storage.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
+RELOCATE_SOURCES = ["head_wise_sparse_b200/csrc/rope.cu", "head_wise_sparse_b200/csrc/device_common.cuh"]
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -384,7 +385,8 @@ def bench_headline(args, torch, dev, stream, barrier, max_over_ranks, world, pk,
                 "queries": f"{T} tokens x {w.hq} heads x {w.d} (one layer of {HEADLINE})",
                 "l2": "operands of 2.8 GB a call, calls back to back",
                 "roofline": roofline(rel_b / (t_rel * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
-                                     "relocate_q_kernel (events around each segkv_relocate_q)")}
+                                     "relocate_q_kernel (events around each segkv_relocate_q)",
+                                     profiled_traffic("relocate_llama70b_layer.md", RELOCATE_SOURCES))}
 
     # ------------------------------------------------------------------ end to end, host buffers
     # every step copies all 4 layers' Q, K and V in from pinned host memory and every layer's
@@ -572,7 +574,8 @@ def bench_mistral(args, torch, dev, stream, max_over_ranks, world, pk):
                        "unit": "GB/s", "ms_per_call": t_rel, "bytes_per_call": rel_b, "calls": n_rel,
                        "l2": "three operand sets in turn (402 MB), calls back to back",
                        "roofline": roofline(rel_b / (t_rel * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
-                                            "relocate_q_kernel (events around each segkv_relocate_q)")}
+                                            "relocate_q_kernel (events around each segkv_relocate_q)",
+                                            profiled_traffic("relocate_mistral7b_8192.md", RELOCATE_SOURCES))}
     del sets
     # attention as a router: every token's received attention mass and the top quarter
     k_top = [L // 4]

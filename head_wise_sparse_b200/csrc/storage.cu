@@ -1,9 +1,8 @@
 // storage.cu -- per-head page tables and the KV append/scatter.
 //
-// The storage itself follows the pages' "per-(layer, head) segmented paged KV storage that
-// physically stores only the tokens each head actually needs" (zhichai.net news item,
-// "What Happened", item 3): a global head's page list grows with the sequence; a local
-// head's list is a ring of R slots, so only the last R logical pages are ever stored.
+// Storage per (layer, KV head), holding only the tokens that head reads (zhichai.net news
+// item, "What Happened", item 3): a global head's page list grows with the sequence; a
+// local head's list is a ring of R slots, so only the last R logical pages are ever stored.
 #include <algorithm>
 
 #include "device_common.cuh"

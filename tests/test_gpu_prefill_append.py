@@ -135,3 +135,29 @@ def test_fused_out_of_pages_changes_nothing(torch_cuda):
     torch.cuda.synchronize()
     assert fused.handle.seq_len(0, 0) == 0 and fused.handle.pages_used == 0
     assert (fused.page_table.cpu().numpy() == -1).all()
+
+
+def test_fused_full_size_mistral_shaped_equals_two_calls(torch_cuda):
+    # the Mistral-shaped step at full size (8 192 tokens, Hq 32, Hkv 8, D 128, 1 global + 7
+    # local W 1024): every CTA stores pages while it attends them
+    torch = torch_cuda
+    from head_wise_sparse_b200.segkv import SegKV
+
+    w = wl.CONFIGS["mistral7b_prefill_L8192"]
+    L = w.seqs[0].length
+    kw = dict(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=w.page, window=w.window,
+              head_class=w.class_array(), num_pages=w.num_pages, free_list=w.free_list(), max_seqs=1,
+              max_seq_len=w.max_seq_len, ring_pages=w.ring_pages, max_chunk=L, ws_batch=1, ws_tokens=L)
+    two, fused = SegKV(**kw), SegKV(**kw)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(66)
+    q = torch.randn((L, w.hq, w.d), generator=g, device="cuda").to(torch.bfloat16)
+    k = (torch.randn((L, w.hkv, w.d), generator=g, device="cuda") / np.sqrt(w.d)).to(torch.bfloat16)
+    v = torch.randn((L, w.hkv, w.d), generator=g, device="cuda").to(torch.bfloat16)
+    vt = torch.zeros((1, w.hq), dtype=torch.int64, device="cuda")
+    vf = torch.zeros((1, w.hq), dtype=torch.int64, device="cuda")
+    two.append(0, [0], [0], [L], k, v)
+    out_t, lse_t = two.prefill(0, [0], [0], [L], q, visited=vt)
+    out_f, lse_f = fused.prefill_append(0, [0], [0], [L], q, k, v, visited=vf)
+    check_same(torch, two, fused)
+    assert torch.equal(out_t, out_f) and torch.equal(lse_t, lse_f) and torch.equal(vt, vf)

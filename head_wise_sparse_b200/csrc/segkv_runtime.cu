@@ -8,9 +8,14 @@
 // kernels.  It never allocates device memory.
 #include <cudaTypedefs.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
-#include <random>
+#include <chrono>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <random>
 #include <cstring>
 #include <new>
 #include <string>
@@ -459,7 +464,42 @@ namespace {
 int noalloc_scratch(segkv_t *h, void **ptr);
 }
 
-int segkv_create(const segkv_config *c, segkv_t **out) {
+}  // extern "C" (the tracing helper below is a template)
+
+// ---------------------------------------------------------------------------- call tracing
+// Every entry point that enqueues work or can fail runs through traced():
+//   SEGKV_LOG=1   one stderr line for each call that returns an error (status, and the
+//                 handle's last CUDA error text when there is one);
+//   SEGKV_LOG=2   one stderr line for every call, with its host time;
+//   SEGKV_NVTX=1  an NVTX range named after the entry point around the call (seen by
+//                 profilers that record NVTX; the NVTX headers load nothing otherwise).
+// Both variables are read once, at the first call.
+namespace {
+int env_level(const char *name) {
+  const char *v = std::getenv(name);
+  return v ? std::atoi(v) : 0;
+}
+template <class F>
+int traced(const char *name, const segkv_t *h, F &&call) {
+  static const int log = env_level("SEGKV_LOG");
+  static const bool nvtx = env_level("SEGKV_NVTX") != 0;
+  if (nvtx) nvtxRangePushA(name);
+  const auto t0 = std::chrono::steady_clock::now();
+  const int rc = call();
+  const double us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
+  if (nvtx) nvtxRangePop();
+  if (log >= 2 || (log >= 1 && rc != SEGKV_OK)) {
+    const bool detail = rc == SEGKV_ERR_CUDA && h && !h->last_error.empty();
+    std::fprintf(stderr, "[segkv] %s -> %d (%s)%s%s, %.1f us on the host\n", name, rc, segkv_strerror(rc),
+                 detail ? ": " : "", detail ? h->last_error.c_str() : "", us);
+  }
+  return rc;
+}
+}  // namespace
+
+extern "C" {
+
+static int segkv_create_impl(const segkv_config *c, segkv_t **out) {
   if (!c || !out) return SEGKV_ERR_INVALID_ARG;
   *out = nullptr;
   if (c->num_layers < 1 || c->num_q_heads < 1 || c->num_kv_heads < 1 || c->max_seqs < 1 || c->max_seq_len < 1 ||
@@ -508,6 +548,9 @@ int segkv_create(const segkv_config *c, segkv_t **out) {
   *out = h;
   return SEGKV_OK;
 }
+int segkv_create(const segkv_config *c, segkv_t **out) {
+  return traced("segkv_create", nullptr, [&] { return segkv_create_impl(c, out); });
+}
 
 void segkv_destroy(segkv_t *h) {
   if (!h) return;
@@ -522,7 +565,7 @@ void segkv_destroy(segkv_t *h) {
 int segkv_ring_pages(const segkv_t *h) { return h ? h->ring : -1; }
 const char *segkv_last_error(const segkv_t *h) { return h ? h->last_error.c_str() : "no handle"; }
 
-int segkv_debug_set(segkv_t *h, int key, long long value) {
+static int segkv_debug_set_impl(segkv_t *h, int key, long long value) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   switch (key) {
     case SEGKV_DEBUG_WAIT_LIMIT:
@@ -540,6 +583,9 @@ int segkv_debug_set(segkv_t *h, int key, long long value) {
     default:
       return SEGKV_ERR_INVALID_ARG;
   }
+}
+int segkv_debug_set(segkv_t *h, int key, long long value) {
+  return traced("segkv_debug_set", h, [&] { return segkv_debug_set_impl(h, key, value); });
 }
 int segkv_max_lp(const segkv_t *h) { return h ? h->max_lp : -1; }
 int segkv_pages_used(const segkv_t *h) { return h ? (int)h->pages_used : -1; }
@@ -574,7 +620,7 @@ size_t segkv_workspace_bytes(const segkv_t *h, int max_batch, int max_tokens) {
   return align_up(std::max(std::max(app, rt), std::max(pre, dec)), 256);
 }
 
-int segkv_reset(segkv_t *h, void *stream) {
+static int segkv_reset_impl(segkv_t *h, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   SEGKV_CUDA(h, "reset launch", launch_reset(geom(h), h->cfg.num_layers, static_cast<cudaStream_t>(stream)));
   std::fill(h->len.begin(), h->len.end(), 0);
@@ -584,8 +630,11 @@ int segkv_reset(segkv_t *h, void *stream) {
   h->pages_used = 0;
   return SEGKV_OK;
 }
+int segkv_reset(segkv_t *h, void *stream) {
+  return traced("segkv_reset", h, [&] { return segkv_reset_impl(h, stream); });
+}
 
-int segkv_fork(segkv_t *h, int src_seq, int dst_seq, void *stream) {
+static int segkv_fork_impl(segkv_t *h, int src_seq, int dst_seq, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   const segkv_config &c = h->cfg;
   if (src_seq < 0 || dst_seq < 0 || src_seq >= c.max_seqs || dst_seq >= c.max_seqs || src_seq == dst_seq)
@@ -610,8 +659,11 @@ int segkv_fork(segkv_t *h, int src_seq, int dst_seq, void *stream) {
   }
   return SEGKV_OK;
 }
+int segkv_fork(segkv_t *h, int src_seq, int dst_seq, void *stream) {
+  return traced("segkv_fork", h, [&] { return segkv_fork_impl(h, src_seq, dst_seq, stream); });
+}
 
-int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *start_pos,
+static int segkv_append_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *start_pos,
                  const int32_t *num_new, const void *k_new, const void *v_new, void *ws, size_t ws_bytes,
                  void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
@@ -758,8 +810,13 @@ int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const 
   h->pages_used += new_pages;
   return SEGKV_OK;
 }
+int segkv_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *start_pos,
+                 const int32_t *num_new, const void *k_new, const void *v_new, void *ws, size_t ws_bytes,
+                 void *stream) {
+  return traced("segkv_append", h, [&] { return segkv_append_impl(h, layer, nseq, seq_ids, start_pos, num_new, k_new, v_new, ws, ws_bytes, stream); });
+}
 
-int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_start_pos, const int32_t *q_len,
+static int segkv_plan_prefill_impl(const segkv_t *h, int layer, int nseq, const int32_t *q_start_pos, const int32_t *q_len,
                        int32_t *items_out, int64_t cap, int64_t *n_items, int *tile_pos, int *key_tile) {
   if (!h || layer < 0 || layer >= h->cfg.num_layers || nseq < 1 || !q_start_pos || !q_len)
     return SEGKV_ERR_INVALID_ARG;
@@ -778,6 +835,10 @@ int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_s
     items_out[4 * i + 3] = items[i].cost;
   }
   return SEGKV_OK;
+}
+int segkv_plan_prefill(const segkv_t *h, int layer, int nseq, const int32_t *q_start_pos, const int32_t *q_len,
+                       int32_t *items_out, int64_t cap, int64_t *n_items, int *tile_pos, int *key_tile) {
+  return traced("segkv_plan_prefill", h, [&] { return segkv_plan_prefill_impl(h, layer, nseq, q_start_pos, q_len, items_out, cap, n_items, tile_pos, key_tile); });
 }
 
 // Prefill, one-source (k_chunk == NULL: every key from the pages) or two-source (the keys of
@@ -966,14 +1027,19 @@ static int prefill_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
   return SEGKV_OK;
 }
 
-int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+static int segkv_prefill_attn_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
                        const int32_t *q_len, const void *q, float softmax_scale, void *out, float *lse,
                        uint64_t *visited, void *ws, size_t ws_bytes, void *stream) {
   return prefill_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, nullptr, nullptr, softmax_scale, out, lse,
                       visited, ws, ws_bytes, stream);
 }
+int segkv_prefill_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                       const int32_t *q_len, const void *q, float softmax_scale, void *out, float *lse,
+                       uint64_t *visited, void *ws, size_t ws_bytes, void *stream) {
+  return traced("segkv_prefill_attn", h, [&] { return segkv_prefill_attn_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, softmax_scale, out, lse, visited, ws, ws_bytes, stream); });
+}
 
-int segkv_prefill_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+static int segkv_prefill_append_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
                          const int32_t *q_len, const void *q, const void *k_new, const void *v_new,
                          float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws, size_t ws_bytes,
                          void *stream) {
@@ -981,8 +1047,14 @@ int segkv_prefill_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids
   return prefill_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, k_new, v_new, softmax_scale, out, lse,
                       visited, ws, ws_bytes, stream, true);
 }
+int segkv_prefill_append(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                         const int32_t *q_len, const void *q, const void *k_new, const void *v_new,
+                         float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws, size_t ws_bytes,
+                         void *stream) {
+  return traced("segkv_prefill_append", h, [&] { return segkv_prefill_append_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, k_new, v_new, softmax_scale, out, lse, visited, ws, ws_bytes, stream); });
+}
 
-int segkv_prefill_attn_2src(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+static int segkv_prefill_attn_2src_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
                             const int32_t *q_len, const void *q, const void *k_chunk, const void *v_chunk,
                             float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws,
                             size_t ws_bytes, void *stream) {
@@ -990,15 +1062,26 @@ int segkv_prefill_attn_2src(segkv_t *h, int layer, int nseq, const int32_t *seq_
   return prefill_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, k_chunk, v_chunk, softmax_scale, out, lse,
                       visited, ws, ws_bytes, stream);
 }
+int segkv_prefill_attn_2src(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                            const int32_t *q_len, const void *q, const void *k_chunk, const void *v_chunk,
+                            float softmax_scale, void *out, float *lse, uint64_t *visited, void *ws,
+                            size_t ws_bytes, void *stream) {
+  return traced("segkv_prefill_attn_2src", h, [&] { return segkv_prefill_attn_2src_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, k_chunk, v_chunk, softmax_scale, out, lse, visited, ws, ws_bytes, stream); });
+}
 
-int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,
+static int segkv_decode_attn_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,
                       const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
                       void *ws, size_t ws_bytes, void *stream) {
   return decode_common(h, layer, nseq, seq_ids, q_pos, q, softmax_scale, num_splits, out, lse, visited, ws, ws_bytes,
                        stream, nullptr);
 }
+int segkv_decode_attn(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_pos,
+                      const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
+                      void *ws, size_t ws_bytes, void *stream) {
+  return traced("segkv_decode_attn", h, [&] { return segkv_decode_attn_impl(h, layer, nseq, seq_ids, q_pos, q, softmax_scale, num_splits, out, lse, visited, ws, ws_bytes, stream); });
+}
 
-int segkv_decode_step(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const void *k_new, const void *v_new,
+static int segkv_decode_step_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const void *k_new, const void *v_new,
                       const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
                       void *ws, size_t ws_bytes, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
@@ -1053,8 +1136,13 @@ int segkv_decode_step(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
   h->pages_used += new_pages;
   return SEGKV_OK;
 }
+int segkv_decode_step(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const void *k_new, const void *v_new,
+                      const void *q, float softmax_scale, int num_splits, void *out, float *lse, uint64_t *visited,
+                      void *ws, size_t ws_bytes, void *stream) {
+  return traced("segkv_decode_step", h, [&] { return segkv_decode_step_impl(h, layer, nseq, seq_ids, k_new, v_new, q, softmax_scale, num_splits, out, lse, visited, ws, ws_bytes, stream); });
+}
 
-int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+static int segkv_router_topk_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
                       const int32_t *q_len, const void *q, const float *lse, float softmax_scale, const int32_t *k,
                       float *scores, int32_t *rows_out, void *ws, size_t ws_bytes, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
@@ -1183,8 +1271,13 @@ int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, c
                          nseq, *std::max_element(q_len, q_len + nseq), scores, rows_out, st));
   return SEGKV_OK;
 }
+int segkv_router_topk(segkv_t *h, int layer, int nseq, const int32_t *seq_ids, const int32_t *q_start_pos,
+                      const int32_t *q_len, const void *q, const float *lse, float softmax_scale, const int32_t *k,
+                      float *scores, int32_t *rows_out, void *ws, size_t ws_bytes, void *stream) {
+  return traced("segkv_router_topk", h, [&] { return segkv_router_topk_impl(h, layer, nseq, seq_ids, q_start_pos, q_len, q, lse, softmax_scale, k, scores, rows_out, ws, ws_bytes, stream); });
+}
 
-int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, const void *q_in, void *q_out,
+static int segkv_relocate_q_impl(segkv_t *h, int layer, int n_tokens, const int32_t *shift, const void *q_in, void *q_out,
                      float theta_base, int interleaved, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   if (layer < 0 || layer >= h->cfg.num_layers || n_tokens < 0 || !(theta_base > 1.0f) ||
@@ -1211,8 +1304,12 @@ int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, 
   SEGKV_CUDA(h, "relocate launch", launch_relocate_q(p, n_tokens, static_cast<cudaStream_t>(stream)));
   return SEGKV_OK;
 }
+int segkv_relocate_q(segkv_t *h, int layer, int n_tokens, const int32_t *shift, const void *q_in, void *q_out,
+                     float theta_base, int interleaved, void *stream) {
+  return traced("segkv_relocate_q", h, [&] { return segkv_relocate_q_impl(h, layer, n_tokens, shift, q_in, q_out, theta_base, interleaved, stream); });
+}
 
-int segkv_device_status(segkv_t *h, void *stream) {
+static int segkv_device_status_impl(segkv_t *h, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t word = 0;
@@ -1221,6 +1318,9 @@ int segkv_device_status(segkv_t *h, void *stream) {
   SEGKV_CUDA(h, "status clear", cudaMemsetAsync(h->cfg.state + 1, 0, sizeof(int32_t), st));
   SEGKV_CUDA(h, "status sync", cudaStreamSynchronize(st));
   return word;
+}
+int segkv_device_status(segkv_t *h, void *stream) {
+  return traced("segkv_device_status", h, [&] { return segkv_device_status_impl(h, stream); });
 }
 
 }  // extern "C"
@@ -1262,7 +1362,7 @@ int noalloc_scratch(segkv_t *h, void **ptr) {
 
 }  // namespace
 
-extern "C" int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
+static int segkv_decode_attn_noalloc_impl(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
                                          const int32_t *q_pos, const void *q, float softmax_scale, int num_splits,
                                          void *out, float *lse, uint64_t *visited, void *stream) {
   if (!h) return SEGKV_ERR_INVALID_ARG;
@@ -1376,4 +1476,9 @@ extern "C" int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const 
   p.newk = nullptr;  // a plain decode: no token to append
   SEGKV_CUDA(h, "decode launch", launch_decode(p, h->kmap, h->vmap, st));
   return SEGKV_OK;
+}
+extern "C" int segkv_decode_attn_noalloc(segkv_t *h, int layer, int nseq, const int32_t *seq_ids,
+                                         const int32_t *q_pos, const void *q, float softmax_scale, int num_splits,
+                                         void *out, float *lse, uint64_t *visited, void *stream) {
+  return traced("segkv_decode_attn_noalloc", h, [&] { return segkv_decode_attn_noalloc_impl(h, layer, nseq, seq_ids, q_pos, q, softmax_scale, num_splits, out, lse, visited, stream); });
 }

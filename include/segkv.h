@@ -31,6 +31,12 @@
  *     never trap.
  *   - A handle is not thread-safe.  Calls on one handle must be issued from one host
  *     thread, in stream order.
+ *   - Tracing, read from the environment at the first call: SEGKV_LOG=1 writes one line to
+ *     stderr for every call that returns an error, SEGKV_LOG=2 one line for every call
+ *     (entry point, status, host time); SEGKV_NVTX=1 wraps every call in an NVTX range
+ *     named after the entry point.  The entry points traced are those that can fail:
+ *     create, reset, fork, append, the prefill, decode, router and relocation calls,
+ *     segkv_device_status and segkv_debug_set.
  */
 #ifndef SEGKV_H_
 #define SEGKV_H_

@@ -203,3 +203,40 @@ def test_binding_argument_counts_match_the_header():
         argtypes = getattr(lib, name).argtypes
         if argtypes is not None:
             assert len(argtypes) == n, (name, len(argtypes), n)
+
+
+LOG_SCRIPT = """
+import sys
+sys.path.insert(0, {root!r})
+from tests.test_abi_host import handle, FAKE
+h = handle(num_pages=20)
+print("rc", h.append(0, [0], [5], [10], FAKE, FAKE, FAKE, 1 << 20, stream=0))
+print("rc", h.seq_len(0, 0))
+print("rc", h.append(1, [0], [0], [1], FAKE, FAKE, FAKE, 1 << 20, stream=0))
+"""
+
+
+def run_logged(env_value):
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ)
+    env.pop("SEGKV_LOG", None)
+    if env_value is not None:
+        env["SEGKV_LOG"] = env_value
+    r = subprocess.run([sys.executable, "-c", LOG_SCRIPT.format(root=root)], capture_output=True, text=True, env=env,
+                       timeout=120)
+    assert r.returncode == 0, r.stderr
+    return r.stdout, [l for l in r.stderr.splitlines() if l.startswith("[segkv]")]
+
+
+def test_log_switch_reports_failed_calls_and_every_call():
+    out, lines = run_logged(None)  # default: silent
+    assert "rc 1" in out and lines == []
+    out, lines = run_logged("1")  # failures only: an append past the stored length, one on a bad layer
+    assert len(lines) == 2 and all(l.startswith("[segkv] segkv_append -> 1 (invalid argument") for l in lines)
+    out, lines = run_logged("2")  # every logged entry point, in order (seq_len is a plain query)
+    assert [l.split()[1] for l in lines] == ["segkv_create", "segkv_append", "segkv_append"]
+    assert lines[0].startswith("[segkv] segkv_create -> 0 (ok")
+    assert all("us on the host" in l for l in lines)

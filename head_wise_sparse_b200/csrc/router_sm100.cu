@@ -132,7 +132,12 @@ __device__ __forceinline__ void router_producer(const CUtensorMap &qmap, const C
       bar->sched[slot] = idx;
       mbar_arrive(&bar->sched_full[slot]);
     }
-    if (idx < 0) break;
+    if (idx < 0) {
+      // no item left for this CTA: the partial-sum kernel may start its CTAs (they wait for
+      // this grid to complete before reading the partials)
+      if (lane == 0) pdl_launch_dependents();
+      break;
+    }
     const RItem it = decode_ritem(p, seqs, items, idx);
     const int kb = i & 1;  // K buffer of this item
     if (!(ok = warp_wait(&bar->k_empty[kb], ((i >> 1) & 1) ^ 1, abort_flag, state))) break;
@@ -445,8 +450,12 @@ __device__ __forceinline__ uint32_t block_scan_excl(uint32_t v, uint32_t *warp_t
   return r;
 }
 
+// Launched as a programmatic dependent of the router kernel, and top-k as one of this kernel:
+// each waits for its primary grid's memory before reading it.
 __global__ void __launch_bounds__(64) score_sum_kernel(const float *__restrict__ part, int slots, int hkv,
                                                       int n_tokens, float *__restrict__ scores) {
+  pdl_launch_dependents();  // top-k may start its CTAs; it waits for this grid to complete
+  pdl_wait_primary();       // the router kernel's partials are complete and visible
   const int t = blockIdx.x * 64 + threadIdx.x;
   if (t >= n_tokens) return;
   const int n = slots * hkv;  // partial j = (slot, head) at part[j * n_tokens + t]
@@ -476,6 +485,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const int4 *__restri
   const int row0 = m.x, n = m.y, k = m.z, out0 = m.w;
   const int tid = threadIdx.x;
   if (k <= 0) return;
+  pdl_wait_primary();  // the scores of score_sum_kernel are complete and visible
   const float *scores = scores_g + row0;
   if (n <= cache_cap) {
     for (int t = tid; t < n; t += kTopkThreads) cache[t] = scores[t];
@@ -534,18 +544,29 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const int4 *__restri
     __syncthreads();
   }
   const uint32_t thr = prefix, need_eq = remaining;  // take every score above thr, need_eq equal to it
-  uint32_t gt_before = 0, eq_before = 0;
-  for (int base = 0; base < n; base += kTopkThreads) {
-    const int t = base + tid;
-    const uint32_t u = t < n ? __float_as_uint(scores[t]) : 0u;
-    const uint32_t gt = (t < n && u > thr) ? 1u : 0u, eq = (t < n && u == thr) ? 1u : 0u;
-    uint32_t total;
-    const uint32_t ex = block_scan_excl(gt | (eq << 16), warp_tot, total);
-    const uint32_t gtb = gt_before + (ex & 0xFFFFu), eqb = eq_before + (ex >> 16);
-    if (gt) rows_out[out0 + gtb + min(eqb, need_eq)] = row0 + t;
-    else if (eq && eqb < need_eq) rows_out[out0 + gtb + eqb] = row0 + t;
-    gt_before += total & 0xFFFFu;
-    eq_before += total >> 16;
+  // thread tid owns the contiguous run [tid * per, tid * per + per): count its scores above
+  // and at the threshold, one block scan of both counts, then write the run's rows in order
+  // (a score above the threshold lands after every selected row before it; an equal one
+  // only while fewer than need_eq equal ones came before it)
+  const int per = (n + kTopkThreads - 1) / kTopkThreads, t0 = tid * per, t1 = min(t0 + per, n);
+  uint32_t gt = 0, eq = 0;
+  for (int t = t0; t < t1; ++t) {
+    const uint32_t u = __float_as_uint(scores[t]);
+    gt += u > thr ? 1u : 0u;
+    eq += u == thr ? 1u : 0u;
+  }
+  uint32_t gt_total, eq_total;
+  uint32_t gtb = block_scan_excl(gt, warp_tot, gt_total);
+  uint32_t eqb = block_scan_excl(eq, warp_tot, eq_total);
+  for (int t = t0; t < t1; ++t) {
+    const uint32_t u = __float_as_uint(scores[t]);
+    if (u > thr) {
+      rows_out[out0 + gtb + min(eqb, need_eq)] = row0 + t;
+      ++gtb;
+    } else if (u == thr) {
+      if (eqb < need_eq) rows_out[out0 + gtb + eqb] = row0 + t;
+      ++eqb;
+    }
   }
 }
 
@@ -574,8 +595,16 @@ cudaError_t launch_router(const RouterLaunch &p, const CUtensorMap &qmap, const 
 
 cudaError_t launch_topk(const float *part, int chunks, int hkv, int n_tokens, const int4 *topk_meta, int nseq,
                         int max_len, float *scores, int32_t *rows_out, cudaStream_t st) {
-  score_sum_kernel<<<(n_tokens + 63) / 64, 64, 0, st>>>(part, chunks, hkv, n_tokens, scores);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((n_tokens + 63) / 64);
+  cfg.blockDim = dim3(64);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, score_sum_kernel, part, chunks, hkv, n_tokens, scores);
   if (e != cudaSuccess) return e;
   // keep up to 16 384 scores (64 KiB) of a sequence in shared memory
   constexpr int kCacheCap = 16384;
@@ -585,8 +614,10 @@ cudaError_t launch_topk(const float *part, int chunks, int hkv, int n_tokens, co
     attr_set = true;
   }
   const int cap = std::min(max_len, kCacheCap);
-  topk_kernel<<<nseq, kTopkThreads, 4 * cap, st>>>(topk_meta, scores, rows_out, cap);
-  return cudaGetLastError();
+  cfg.gridDim = dim3(nseq);
+  cfg.blockDim = dim3(kTopkThreads);
+  cfg.dynamicSmemBytes = 4 * cap;
+  return cudaLaunchKernelEx(&cfg, topk_kernel, topk_meta, static_cast<const float *>(scores), rows_out, cap);
 }
 
 }  // namespace skv

@@ -89,6 +89,21 @@ def test_gqa_groups_and_ragged_lengths(torch_cuda, g):
     check_against_oracle(w, 0, q, out, lse, vis, ids, qs, ql)
 
 
+# edge configurations: a window of one key (each query sees only itself on a local head), 16
+# query heads a KV head (8 positions a 128-row tile), a layer whose heads are all local and
+# one whose heads are all global; ragged lengths that end mid-tile and mid-page
+@pytest.mark.parametrize("name,g,window,cls", [("w1", 2, 1, (1, 0)), ("g16", 16, 100, (0, 1)),
+                                               ("all_local", 4, 64, (0, 0)), ("all_global", 4, 64, (1, 1))])
+def test_edge_windows_groups_and_classes(torch_cuda, name, g, window, cls):
+    hkv = 2
+    seqs = (Seq(0, 333, 0, 333), Seq(0, 70, 0, 70), Seq(0, 1, 0, 1))
+    w = Workload(340 + g + window, name, 1, hkv * g, hkv, 128, 16, window, 64, seqs, (cls,))
+    kv, q, out, lse, vis = run_prefill_case(torch_cuda, w)
+    ids, qs, ql = step_queries(w)
+    o = check_against_oracle(w, 0, q, out, lse, vis, ids, qs, ql)
+    assert np.array_equal(kv.page_table.cpu().numpy(), o.page_table())
+
+
 def test_mistral_shape_scaled_length(torch_cuda):
     w = wl.CONFIGS["mistral7b_prefill_L8192"].scaled(seqs=(Seq(0, 2048, 0, 2048),), ring_pages=32)
     kv, q, out, lse, vis = run_prefill_case(torch_cuda, w)

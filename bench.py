@@ -460,7 +460,9 @@ def bench_headline(args, torch, dev, stream, barrier, max_over_ranks, world, pk,
                              frac_of_sustained=achieved / pk["bf16_tflops_sustained"]),
         "append": {"bytes": app_b, "ms": t_app, "GB/s": app_b / (t_app * 1e-3) / 1e9,
                    "roofline": roofline(app_b / (t_app * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm",
-                                        "reset_kernel + append_kernel x 4 (events around reset + the 4 segkv_append calls)")},
+                                        "reset_kernel + append_kernel x 4 (events around reset + the 4 segkv_append calls)",
+                                        profiled_traffic("append_llama70b_layer.md", APPEND_SOURCES),
+                                        traffic_per="append_kernel launch (one layer)")},
         "config": {"workload": HEADLINE, "layers": L, "seq_lens": lens, "q_heads": w.hq, "kv_heads": w.hkv,
                    "head_dim": w.d, "page_size": w.page, "window": w.window,
                    "global_kv_heads_per_layer": [int(sum(c)) for c in w.classes],

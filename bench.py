@@ -645,6 +645,44 @@ def bench_tiny(args, torch, dev, stream, max_over_ranks, world, pk):
             "gpu_launches": len(ev)}
 
 
+def bench_headline_slice(args, torch, dev, stream, max_over_ranks, world, pk):
+    """The headline's prefill kernel on a slice small enough for a full ncu capture (the
+    profiling leg): one layer of the Llama-shaped heads (Hq 64, Hkv 8, D 128, W 2048, layer
+    0's head classes) over one sequence of 8 192 tokens -- 134 MB of Q, more than L2, under
+    1 GB on the device."""
+    base = wl.CONFIGS[HEADLINE]
+    w = base.scaled(layers=1, classes=base.classes[:1], seqs=(wl.Seq(0, 8192, 0, 8192),))
+    L = 8192
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(17)
+    q = torch.randn((L, w.hq, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    k = torch.randn((L, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    v = torch.randn((L, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((L, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((L, w.hq), dtype=torch.float32, device=dev)
+    kv = new_handle(w, dev, ws_tokens=L, max_chunk=L)
+    kv.append(0, [0], [0], [L], k, v)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    times = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kv.prefill(0, [0], [0], [L], q, out=out, lse=lse)
+        e1.record(stream)
+        if i >= args.warmup:
+            times.append((e0, e1))
+    torch.cuda.synchronize()
+    if kv.device_status() != 0:
+        raise RuntimeError("device error word set during the headline slice")
+    t = max_over_ranks(sum(a.elapsed_time(b) for a, b in times) / len(times))
+    flops = 4.0 * w.d * visible_pairs(w)
+    del kv, q, k, v, out, lse, flush
+    torch.cuda.empty_cache()
+    return {"workload": "llama70b_layer0_heads_one_sequence_8192", "ms": t, "TFLOP/s": flops / (t * 1e-3) / 1e12,
+            "frac": flops / (t * 1e-3) / 1e12 / pk["bf16_tflops"]}
+
+
 def bench_append_layer(args, torch, dev, stream, max_over_ranks, world, pk):
     """The append of one Llama-shaped layer (4 sequences of the seeded lengths, Hkv 8, D 128,
     181 MB of K/V read and written) into an emptied handle, alone (the profiling leg)."""
@@ -689,9 +727,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", default="", choices=["", "headline", "mistral", "chunked", "tiny", "fork", "decode",
-                                                   "append"],
+                                                   "append", "headline_slice"],
                     help="run one leg alone (for profiling): the headline step, or one sub-workload; 'append' is the "
-                         "append of one Llama-shaped layer (181 MB of K/V, about 1 GB on the device)")
+                         "append of one Llama-shaped layer (181 MB of K/V, about 1 GB on the device); "
+                         "'headline_slice' the headline's prefill kernel on one 8 192-token sequence of its heads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -721,7 +760,8 @@ def main():
                 "tiny": lambda: bench_tiny(args, torch, dev, stream, max_over_ranks, world, pk),
                 "fork": lambda: bench_fork(args, torch, dev, stream, max_over_ranks, world, pk),
                 "decode": lambda: bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk),
-                "append": lambda: bench_append_layer(args, torch, dev, stream, max_over_ranks, world, pk)}
+                "append": lambda: bench_append_layer(args, torch, dev, stream, max_over_ranks, world, pk),
+                "headline_slice": lambda: bench_headline_slice(args, torch, dev, stream, max_over_ranks, world, pk)}
         res = legs[args.only]()
         sampler.stop()
         if world > 1:

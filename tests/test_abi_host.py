@@ -216,15 +216,18 @@ print("rc", h.append(1, [0], [0], [1], FAKE, FAKE, FAKE, 1 << 20, stream=0))
 """
 
 
-def run_logged(env_value):
+def run_logged(env_value, nvtx=False):
     import subprocess
     import sys
 
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     env = dict(os.environ)
     env.pop("SEGKV_LOG", None)
+    env.pop("SEGKV_NVTX", None)
     if env_value is not None:
         env["SEGKV_LOG"] = env_value
+    if nvtx:
+        env["SEGKV_NVTX"] = "1"  # ranges are pushed and popped; without a profiler they cost nothing
     r = subprocess.run([sys.executable, "-c", LOG_SCRIPT.format(root=root)], capture_output=True, text=True, env=env,
                        timeout=120)
     assert r.returncode == 0, r.stderr
@@ -236,7 +239,9 @@ def test_log_switch_reports_failed_calls_and_every_call():
     assert "rc 1" in out and lines == []
     out, lines = run_logged("1")  # failures only: an append past the stored length, one on a bad layer
     assert len(lines) == 2 and all(l.startswith("[segkv] segkv_append -> 1 (invalid argument") for l in lines)
-    out, lines = run_logged("2")  # every logged entry point, in order (seq_len is a plain query)
-    assert [l.split()[1] for l in lines] == ["segkv_create", "segkv_append", "segkv_append"]
-    assert lines[0].startswith("[segkv] segkv_create -> 0 (ok")
-    assert all("us on the host" in l for l in lines)
+    for nvtx in (False, True):
+        out, lines = run_logged("2", nvtx)  # every logged entry point, in order (seq_len is a plain query)
+        assert out.split() == ["rc", "1", "rc", "0", "rc", "1"]
+        assert [l.split()[1] for l in lines] == ["segkv_create", "segkv_append", "segkv_append"]
+        assert lines[0].startswith("[segkv] segkv_create -> 0 (ok")
+        assert all("us on the host" in l for l in lines)

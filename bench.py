@@ -899,48 +899,67 @@ def bench_chunked(args, torch, dev, stream, max_over_ranks, world, pk):
 
 def bench_fork(args, torch, dev, stream, max_over_ranks, world, pk):
     """Copy on write after a fork: 64 sequences of 1000 tokens (Mistral-shaped heads) are
-    forked into 64 empty slots; the timed call appends one token to every fork, so each of
-    the 8 heads of each fork first copies its shared, partly filled last page (the rows
-    before the new token) into a fresh page.  Bytes: the copied rows plus the new rows."""
+    forked into 8 groups of 64 empty slots; each timed call appends one token to every fork
+    of one group, so each of the 8 heads of each fork first copies its shared, partly filled
+    last page (the rows before the new token) into a fresh page.  The 8 calls of a step run
+    back to back after a sleep kernel lets the host queue them (the events time the GPU's
+    work); one call on an idle GPU, host planning included, is reported beside it.  Bytes:
+    the copied rows plus the new rows, read and written."""
     from head_wise_sparse_b200.segkv import SegKV
 
     w = wl.CONFIGS[PREFILL]
-    B, ctx, P = 64, 1000, w.page
-    n_pages = 2 * B * w.hkv * (ctx // P + 2) + 64
+    B, ctx, P, NG = 64, 1000, w.page, 8
+    n_pages = B * w.hkv * ((ctx // P + 2) + NG) + 64
     free = np.random.default_rng(7).permutation(n_pages).astype(np.int32)
     kv = SegKV(num_layers=1, num_q_heads=w.hq, num_kv_heads=w.hkv, head_dim=w.d, page_size=P, window=w.window,
-               head_class=w.class_array(), num_pages=n_pages, free_list=free, max_seqs=2 * B, max_seq_len=ctx + 8,
-               ring_pages=-(-(ctx + 8) // P), max_chunk=ctx, ws_batch=B, ws_tokens=B * ctx, device=dev)
+               head_class=w.class_array(), num_pages=n_pages, free_list=free, max_seqs=(NG + 1) * B,
+               max_seq_len=ctx + 8, ring_pages=-(-(ctx + 8) // P), max_chunk=ctx, ws_batch=B, ws_tokens=B * ctx,
+               device=dev)
     gen = torch.Generator(device=dev)
     gen.manual_seed(11)
     k = torch.randn((B * ctx, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
     k1 = torch.randn((B, w.hkv, w.d), generator=gen, device=dev).to(torch.bfloat16)
-    src, dst = list(range(B)), list(range(B, 2 * B))
-    times = []
-    for it in range(args.warmup + 10):
+    src = list(range(B))
+    groups = [list(range((g + 1) * B, (g + 2) * B)) for g in range(NG)]
+    queued, idle = [], []
+    for it in range(args.warmup + max(3, min(args.steps, 10))):
         kv.reset()
         kv.append(0, src, [0] * B, [ctx] * B, k, k)
-        for a, b in zip(src, dst):
-            kv.fork(a, b)
+        for grp in groups:
+            for a, b in zip(src, grp):
+                kv.fork(a, b)
+        torch.cuda.synchronize()
+        # one group on an idle GPU, host planning and upload inside the events
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        kv.append(0, dst, [ctx] * B, [1] * B, k1, k1)
+        kv.append(0, groups[0], [ctx] * B, [1] * B, k1, k1)
         e1.record(stream)
         torch.cuda.synchronize()
+        # the other groups back to back, queued behind a sleep kernel
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in groups[1:]]
+        torch.cuda._sleep(2_000_000)
+        for (a, b), grp in zip(evs, groups[1:]):
+            a.record(stream)
+            kv.append(0, grp, [ctx] * B, [1] * B, k1, k1)
+            b.record(stream)
+        torch.cuda.synchronize()
         if it >= args.warmup:
-            times.append(e0.elapsed_time(e1))
+            idle.append(e0.elapsed_time(e1))
+            queued.extend(a.elapsed_time(b) for a, b in evs)
     if kv.device_status() != 0:
         raise RuntimeError("device error word set during the fork benchmark")
-    t = max_over_ranks(statistics.median(times))
+    t = max_over_ranks(statistics.median(queued))
+    t_idle = max_over_ranks(statistics.median(idle))
     moved = B * w.hkv * ((ctx % P) + 1) * w.d * 2 * 2 * 2  # K and V: copied rows read + written, new row
     del kv, k, k1
     torch.cuda.empty_cache()
     return {"metric": "copy-on-write append GB/s", "value": world * moved / (t * 1e-3) / 1e9, "unit": "GB/s",
-            "ms_per_call": t, "bytes_per_call": moved, "pages_copied": B * w.hkv,
-            "step": "append 1 token to 64 forks of 1000-token sequences (8 heads each: 512 shared pages copied)",
+            "ms_per_call": t, "ms_per_call_idle_gpu": t_idle, "bytes_per_call": moved, "pages_copied": B * w.hkv,
+            "step": "append 1 token to 64 forks of 1000-token sequences (8 heads each: 512 shared pages copied); "
+                    "calls back to back over 8 fork groups",
             "roofline": {"bound": "hbm", "achieved": moved / (t * 1e-3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": moved / (t * 1e-3) / 1e9 / pk["hbm_gbs"], "traffic": None,
-                         "kernel": "cow_copy_kernel + append_kernel (events around segkv_append)"}}
+                         "kernel": "append_kernel with the copy on write folded in (events around each segkv_append)"}}
 
 
 def bench_decode(args, torch, dev, stream, barrier, max_over_ranks, world, pk):

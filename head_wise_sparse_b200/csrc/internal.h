@@ -67,11 +67,12 @@ struct StorageGeom {  // what every kernel needs to resolve a logical position t
 // -- launchers (each .cu file exposes one host function per kernel) --------------------
 cudaError_t launch_reset(const StorageGeom &g, int num_layers, cudaStream_t st);
 
-// Copies on write first (n_jobs > 0: jobs_dev[j] = (k_new, k_old, rows)), then the scatter;
-// plan_dev == NULL when no page of the call is shared; max_pages = the most pages the call
-// touches for one (sequence, head).
+// The scatter, with the copy on write of shared pages folded in: plan_dev == NULL when no page
+// of the call is shared; else plan_src_dev[i] = the free-list entry of the shared page whose
+// rows before the call's first token the page of plan entry i copies first, or -1;
+// max_pages = the most pages the call touches for one (sequence, head).
 cudaError_t launch_append(const StorageGeom &g, int layer, const void *ws_meta, int nseq, const uint8_t *cls_dev,
-                          const int32_t *pair_off_dev, const int32_t *plan_dev, const int4 *jobs_dev, int n_jobs,
+                          const int32_t *pair_off_dev, const int32_t *plan_dev, const int32_t *plan_src_dev,
                           int cursor0, int new_pages, int max_pages, const void *k_new, const void *v_new,
                           cudaStream_t st);
 

@@ -698,7 +698,7 @@ static int segkv_append_impl(segkv_t *h, int layer, int nseq, const int32_t *seq
   std::vector<int32_t> pair_page((size_t)nseq * H + 1, 0);  // first plan entry of each pair
   std::vector<int32_t> pair_new((size_t)nseq * H + 1, 0);   // pages allocated for earlier pairs
   std::vector<int32_t> plan;
-  std::vector<int4> jobs;  // (k_new, k_old, rows before the call's first token)
+  std::vector<int32_t> plan_src;  // per plan entry: the shared page to copy rows from, else -1
   const bool copies = h->n_shared > 0;  // else every page is one sequence's: no copy, no plan
   // changes to the mirror, applied once the call is accepted; refcounts seen through them, so
   // a page one sequence of the call copies is no longer shared for a later one
@@ -733,12 +733,13 @@ static int segkv_append_impl(segkv_t *h, int layer, int nseq, const int32_t *seq
         const int32_t k_old = h->slot_k[idx];
         if (k_old >= 0 && ref_of(k_old) <= 1) {
           plan.push_back(-1);
+          plan_src.push_back(-1);
           continue;
         }
         const int32_t k_new = (int32_t)(h->pages_used + new_pages++);
         const int copy_rows = (k_old >= 0 && lp == first / P) ? first % P : 0;
         plan.push_back(k_new);
-        if (copy_rows > 0) jobs.push_back(make_int4(k_new, k_old, copy_rows, 0));
+        plan_src.push_back(copy_rows > 0 ? k_old : -1);
         slot_set.push_back({idx, k_new});
         if (k_old >= 0) {
           if (h->ref_scratch[k_old] == 0) ref_keys.push_back(k_old);
@@ -752,8 +753,8 @@ static int segkv_append_impl(segkv_t *h, int layer, int nseq, const int32_t *seq
   const size_t cls_off = kHeaderBytes + sizeof(AppendSeq) * nseq;
   const size_t off_off = cls_off + align_up(H, 4);
   const size_t plan_off = align_up(off_off + 4 * ((size_t)H * nseq + 1), 16);
-  const size_t jobs_off = align_up(plan_off + 4 * plan.size(), 16);
-  const size_t bytes = jobs_off + sizeof(int4) * jobs.size();
+  const size_t src_off = align_up(plan_off + 4 * plan.size(), 16);
+  const size_t bytes = src_off + 4 * plan_src.size();
   if (!ws || !aligned(ws, 256) || ws_bytes < bytes) return SEGKV_ERR_WORKSPACE;
   if ((rc = ensure_device_state(h))) return rc;
   if (total == 0) return SEGKV_OK;
@@ -769,16 +770,16 @@ static int segkv_append_impl(segkv_t *h, int layer, int nseq, const int32_t *seq
   std::memcpy(static_cast<char *>(host) + cls_off, &h->cls[(size_t)layer * H], H);
   std::memcpy(static_cast<char *>(host) + off_off, copies ? pair_page.data() : pair_new.data(), 4 * pair_page.size());
   if (!plan.empty()) std::memcpy(static_cast<char *>(host) + plan_off, plan.data(), 4 * plan.size());
-  if (!jobs.empty()) std::memcpy(static_cast<char *>(host) + jobs_off, jobs.data(), sizeof(int4) * jobs.size());
+  if (!plan_src.empty()) std::memcpy(static_cast<char *>(host) + src_off, plan_src.data(), 4 * plan_src.size());
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = upload(h, ws, bytes, st))) return rc;
   const uint8_t *cls_dev = static_cast<const uint8_t *>(ws) + cls_off;
   const int32_t *off_dev = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + off_off);
   const int32_t *plan_dev = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + plan_off);
-  const int4 *jobs_dev = reinterpret_cast<const int4 *>(static_cast<const char *>(ws) + jobs_off);
+  const int32_t *src_dev = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + src_off);
   SEGKV_CUDA(h, "append launch",
-             launch_append(geom(h), layer, ws, nseq, cls_dev, off_dev, copies ? plan_dev : nullptr, jobs_dev,
-                           (int)jobs.size(), (int)h->pages_used, (int)new_pages, max_pages, k_new, v_new, st));
+             launch_append(geom(h), layer, ws, nseq, cls_dev, off_dev, copies ? plan_dev : nullptr, src_dev,
+                           (int)h->pages_used, (int)new_pages, max_pages, k_new, v_new, st));
   if (copies) {
     for (const auto &e : slot_set) {
       h->slot_k[e.first] = e.second;

@@ -25,34 +25,6 @@ cudaError_t launch_reset(const StorageGeom &g, int num_layers, cudaStream_t st) 
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------------------- copy on write
-// One thread per (job, row, 16-byte chunk): job j = (k_new, k_old, rows) copies rows
-// [0, rows) of K and V from the page at free-list entry k_old (shared with another sequence
-// after a fork) to the fresh page at entry k_new.  It runs before the append kernel on the
-// same stream; the rows it writes lie before the call's first token on that page, so the
-// two kernels never write the same row.
-__global__ void __launch_bounds__(256) cow_copy_kernel(StorageGeom g, const int4 *__restrict__ jobs,
-                                                       long long total) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= total) return;
-  const int CH = g.head_dim / 8, P = g.page;
-  const int c = (int)(i % CH);
-  const int r = (int)((i / CH) % P);
-  const int4 e = jobs[i / ((long long)CH * P)];
-  if (r >= e.z) return;
-  const int32_t dst = (e.x >= 0 && e.x < g.num_pages) ? g.free_list[e.x] : -1;
-  const int32_t src = (e.y >= 0 && e.y < g.num_pages) ? g.free_list[e.y] : -1;
-  if (dst < 0 || dst >= g.num_pages || src < 0 || src >= g.num_pages) {
-    set_error(g.state, kErrDeviceBounds);
-    return;
-  }
-  uint4 *kp = reinterpret_cast<uint4 *>(g.k_pool);
-  uint4 *vp = reinterpret_cast<uint4 *>(g.v_pool);
-  const long long from = ((long long)src * P + r) * CH + c, to = ((long long)dst * P + r) * CH + c;
-  kp[to] = kp[from];
-  vp[to] = vp[from];
-}
-
 // ---------------------------------------------------------------------------- scatter
 // One warp per (sequence of the call, KV head, logical page the call touches): the warp
 // resolves the page once and then moves the page's rows of K and V with 16-byte loads and
@@ -62,8 +34,13 @@ __global__ void __launch_bounds__(256) cow_copy_kernel(StorageGeom g, const int4
 // earlier (sequence, head) pairs).  Otherwise the host lists every page the call touches, in
 // the allocation order (sequence in call order, head ascending, logical page ascending):
 // plan[pair_off[sequence, head] + (lp - lp0)] = the free-list entry the page takes (its slot
-// was empty, or held a page shared after a fork, whose rows before the call were copied by
-// cow_copy_kernel), or -1 (the slot's page is this sequence's alone: written in place).
+// was empty, or held a page shared after a fork), or -1 (the slot's page is this sequence's
+// alone: written in place); plan_src at the same index = the free-list entry of the shared
+// page whose rows before the call's first token the warp copies first (copy on write), or -1.
+// While a page is shared every sharer has the same length (sharing comes from a fork, and a
+// sharer's first append takes it its own copy), so a sharer that copies the rows before that
+// position and a later sharer of the same call that writes the page in place from it on
+// touch disjoint rows.
 // A local head keeps only the last R pages ending at the call's last token, so pages before
 // them have no warp.  The warp holding the call's last page zeroes the rows after its last
 // token on a page the call started or took, so every stored page holds finite values in
@@ -73,8 +50,8 @@ constexpr int kAppendBatch = 8;  // 16-byte chunks of K (and of V) in flight per
 
 __global__ void __launch_bounds__(32 * kAppendWarps) append_kernel(
     StorageGeom g, int layer, const AppendSeq *__restrict__ seqs, int nseq, const uint8_t *__restrict__ cls,
-    const int32_t *__restrict__ pair_off, const int32_t *__restrict__ plan, int cursor0, int new_pages,
-    const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new) {
+    const int32_t *__restrict__ pair_off, const int32_t *__restrict__ plan, const int32_t *__restrict__ plan_src,
+    int cursor0, int new_pages, const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new) {
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) g.state[0] = cursor0 + new_pages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = g.hkv, P = g.page, R = g.ring, CH = g.head_dim / 8;
@@ -114,25 +91,37 @@ __global__ void __launch_bounds__(32 * kAppendWarps) append_kernel(
       if (lane == 0) set_error(g.state, kErrDeviceBounds);
       continue;
     }
-    const long long src0 = ((long long)s.tok_off + (lp * P + r0 - first)) * H + h;  // source row of row r0
     const long long dst0 = (long long)phys * P;
-    const int n = r1 - r0;
-    for (int base = 0; base < n; base += rows_per_step * kAppendBatch) {
+    // copy on write: rows [0, r0) come from the shared page, in the same pass as the new rows
+    const int ks = plan ? plan_src[pair_off[pair] + (lp - lp0)] : -1;
+    long long old0 = 0;
+    if (ks >= 0) {
+      const int32_t old = ks < g.num_pages ? g.free_list[ks] : -1;
+      if (old < 0 || old >= g.num_pages) {
+        if (lane == 0) set_error(g.state, kErrDeviceBounds);
+        continue;
+      }
+      old0 = (long long)old * P;
+    }
+    const int rb = ks >= 0 ? 0 : r0;  // first row this warp writes
+    const long long src0 = ((long long)s.tok_off + (lp * P - first)) * H + h;  // source row of page row 0
+    for (int base = rb; base < r1; base += rows_per_step * kAppendBatch) {
       uint4 kk[kAppendBatch], vv[kAppendBatch];
 #pragma unroll
       for (int u = 0; u < kAppendBatch; ++u) {
         const int r = base + u * rows_per_step + sub;
-        if (r < n) {
-          kk[u] = k_new[(src0 + (long long)r * H) * CH + c];
-          vv[u] = v_new[(src0 + (long long)r * H) * CH + c];
+        if (r < r1) {
+          const long long from = r < r0 ? (old0 + r) * CH + c : (src0 + (long long)r * H) * CH + c;
+          kk[u] = r < r0 ? kp[from] : k_new[from];
+          vv[u] = r < r0 ? vp[from] : v_new[from];
         }
       }
 #pragma unroll
       for (int u = 0; u < kAppendBatch; ++u) {
         const int r = base + u * rows_per_step + sub;
-        if (r < n) {
-          kp[(dst0 + r0 + r) * CH + c] = kk[u];
-          vp[(dst0 + r0 + r) * CH + c] = vv[u];
+        if (r < r1) {
+          kp[(dst0 + r) * CH + c] = kk[u];
+          vp[(dst0 + r) * CH + c] = vv[u];
         }
       }
     }
@@ -148,20 +137,15 @@ __global__ void __launch_bounds__(32 * kAppendWarps) append_kernel(
 }
 
 cudaError_t launch_append(const StorageGeom &g, int layer, const void *ws_meta, int nseq, const uint8_t *cls_dev,
-                          const int32_t *pair_off_dev, const int32_t *plan_dev, const int4 *jobs_dev, int n_jobs,
+                          const int32_t *pair_off_dev, const int32_t *plan_dev, const int32_t *plan_src_dev,
                           int cursor0, int new_pages, int max_pages, const void *k_new, const void *v_new,
                           cudaStream_t st) {
-  if (n_jobs > 0) {
-    const long long copies = (long long)n_jobs * g.page * (g.head_dim / 8);
-    cow_copy_kernel<<<(int)((copies + 255) / 256), 256, 0, st>>>(g, jobs_dev, copies);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
   const AppendSeq *seqs = reinterpret_cast<const AppendSeq *>(static_cast<const char *>(ws_meta) + kHeaderBytes);
   const dim3 grid((unsigned)std::max(1, (max_pages + kAppendWarps - 1) / kAppendWarps),
                   (unsigned)std::min(std::max(1, nseq * g.hkv), 65535));
-  append_kernel<<<grid, 32 * kAppendWarps, 0, st>>>(g, layer, seqs, nseq, cls_dev, pair_off_dev, plan_dev, cursor0,
-                                                    new_pages, reinterpret_cast<const uint4 *>(k_new),
+  append_kernel<<<grid, 32 * kAppendWarps, 0, st>>>(g, layer, seqs, nseq, cls_dev, pair_off_dev, plan_dev,
+                                                    plan_src_dev, cursor0, new_pages,
+                                                    reinterpret_cast<const uint4 *>(k_new),
                                                     reinterpret_cast<const uint4 *>(v_new));
   return cudaGetLastError();
 }
